@@ -1,0 +1,256 @@
+"""fp64 CPU oracle for the HySparse2 KV Reuse hot path -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and bench.py's CPU-baseline leg may
+import this package.  It shares no code with the CUDA library and never
+imports it; both sides only share the seeded input generator ``synth``.
+
+Everything here is the plain definition of what the method computes, written
+row by row in float64 with numpy (a matmul, an exp, a sort are the only library
+steps).  Sources, by page and passage:
+
+* "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing" (agihunt.info
+  summary), paragraph on inner-level KV Reuse: the full-attention layer scores
+  tokens one by one; the 128 most recent tokens are always put in the sparse
+  selection and 1024 high-scoring out-of-window tokens are added; the sparse
+  layers read the same full-attention KV.
+* same page, next paragraph: MQA (one KV head), NoPE on full and sparse layers,
+  the full layer is an oracle selector using exact attention scores.
+* same page, the outer-level KV Bridging paragraph: a cross-decoder full
+  layer's K/V are the source hidden state re-projected by that layer's own
+  projections.
+* same page, results table header "KV @1M (FP8)": the KV cache is stored FP8.
+* 10100.com article, "evolution two": the selection adds *at most* 1024 tokens.
+
+Readings where the pages are silent (the same readings the CUDA path uses):
+head aggregation = sum over the query heads of the softmax probabilities;
+window = positions [p-W+1, p] (it includes the query itself); candidates =
+[0, p-W]; softmax scale 1/sqrt(d); ties in the score broken by smaller
+position; FP8 = OCP E4M3FN, round-to-nearest-even, saturating at +-448, one
+fp32 scale per token row = amax/448 (1 for an all-zero row).
+
+Parity unpinned (no page fixes it; pinned only to the stated reading): the
+head aggregation rule, the softmax scale and the tie order.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+
+def f64(x) -> np.ndarray:
+    """Any array (numpy, or a CPU torch tensor of any float dtype) as float64."""
+    if hasattr(x, "detach"):
+        import torch
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def u8(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        return x.detach().cpu().numpy().astype(np.uint8, copy=False)
+    return np.asarray(x, dtype=np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3FN (storage format of the KV cache)
+# ---------------------------------------------------------------------------
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3FN code: 1 sign, 4 exponent (bias 7), 3 mantissa bits;
+    exponent field 0 is subnormal (2^-6 * m/8); code 0x7F/0xFF is NaN; no inf."""
+    s = (code >> 7) & 1
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return -v if s else v
+
+
+E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+# non-negative finite codes 0x00..0x7E in increasing value order
+_POS_VALUES = E4M3_TABLE[:0x7F]
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """Nearest E4M3FN code, ties to the even code, |x| >= 448 saturates to 448."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    sign = np.signbit(x).astype(np.uint8) << 7
+    hi = np.searchsorted(_POS_VALUES, a, side="left")          # first value >= a
+    hi = np.minimum(hi, 0x7E)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - _POS_VALUES[lo]
+    dhi = _POS_VALUES[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(a >= E4M3_MAX, 0x7E, code).astype(np.uint8)
+    code = np.where(np.isnan(x), 0x7F, code | sign).astype(np.uint8)
+    return code
+
+
+def quantize_rows_e4m3(X: np.ndarray):
+    """Per-row FP8 storage: scale = amax/448 (1 if amax == 0), code = E4M3(x/scale).
+
+    Returns (codes uint8 [R,d], scales float64 [R], pre-rounding values x/scale).
+    """
+    X = f64(X)
+    amax = np.abs(X).max(axis=1)
+    scale = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    y = X / scale[:, None]
+    return e4m3_encode(y), scale, y
+
+
+# ---------------------------------------------------------------------------
+# KV Bridging
+# ---------------------------------------------------------------------------
+
+def bridge_rows(hidden: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """K_r = sum_c hidden[r,c] * W[:,c]  (W in [out, in] layout), fp64."""
+    return f64(hidden) @ f64(W).T
+
+
+# ---------------------------------------------------------------------------
+# Full attention as the oracle selector, and the index set
+# ---------------------------------------------------------------------------
+
+@dataclass
+class SelectRow:
+    p: int                    # absolute position of the query
+    O: np.ndarray             # [H, d] attention output (unrounded)
+    m: np.ndarray             # [H] row max of the logits
+    l: np.ndarray             # [H] sum of exp(s - m)
+    sigma: np.ndarray         # [p+1] head-summed probabilities
+    idx: np.ndarray           # [window + topk] int32
+    tau: Optional[float]      # k-th largest sigma among candidates (None: all taken)
+    n_sel: int
+
+
+def window_slots(p: int, window: int) -> np.ndarray:
+    """Forced recent window: slot w holds position p-window+1+w, -1 if negative."""
+    pos = np.arange(p - window + 1, p + 1, dtype=np.int64)
+    return np.where(pos >= 0, pos, -1).astype(np.int32)
+
+
+def topk_positions(sigma_c: np.ndarray, k: int) -> np.ndarray:
+    """The k candidates with the largest score, ties to the smaller position,
+    returned in ascending position order (all of them if there are <= k)."""
+    n = sigma_c.shape[0]
+    if n <= k:
+        return np.arange(n, dtype=np.int64)
+    order = np.lexsort((np.arange(n), -sigma_c))   # by -sigma, then position
+    return np.sort(order[:k])
+
+
+def select_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, p: int, window: int,
+               topk: int, scale: float) -> SelectRow:
+    """One query row of the full-attention layer (MQA, NoPE) and its index set.
+
+    q: [H, d] fp64; K, V: [>= p+1, d] fp64 (the single KV head).
+    """
+    s = (q @ K[:p + 1].T) * scale                    # [H, p+1] logits
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    l = e.sum(axis=1)
+    P = e / l[:, None]                               # exact softmax probabilities
+    O = P @ V[:p + 1]                                # [H, d]
+    sigma = P.sum(axis=0)                            # head-summed score per key
+    n_cand = max(0, p - window + 1)                  # candidates 0 .. p-window
+    sel = topk_positions(sigma[:n_cand], topk)
+    tau = None
+    if n_cand > topk:
+        tau = float(np.sort(sigma[:n_cand])[-topk])
+    idx = np.full(window + topk, -1, dtype=np.int32)
+    idx[:window] = window_slots(p, window)
+    idx[window:window + sel.shape[0]] = sel
+    return SelectRow(p, O, m, l, sigma, idx, tau, int(sel.shape[0]))
+
+
+def full_attn_select(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rows: Sequence[int],
+                     q_start: int, window: int, topk: int,
+                     scale: Optional[float] = None) -> Dict[int, SelectRow]:
+    """Prefill: query t sits at absolute position q_start + t and sees keys <= it.
+
+    Q: [Tq, H, d]; K, V: [kv_len, d] -- any float dtype, read as fp64.
+    """
+    d = Q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    K = f64(K)
+    V = f64(V)
+    out = {}
+    for t in rows:
+        q = f64(Q[t])
+        out[t] = select_row(q, K, V, q_start + t, window, topk, scale)
+    return out
+
+
+def sparse_attn_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx_row: np.ndarray,
+                    scale: float) -> np.ndarray:
+    """Sparse layer: softmax attention of its own q over the selected keys only."""
+    S = idx_row[idx_row >= 0].astype(np.int64)
+    s = (q @ K[S].T) * scale                         # [H, |S|]
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    P = e / e.sum(axis=1, keepdims=True)
+    return P @ V[S]
+
+
+def sparse_attn(Qs: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray,
+                rows: Sequence[int], scale: Optional[float] = None) -> Dict[int, np.ndarray]:
+    d = Qs.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    K = f64(K)
+    V = f64(V)
+    idx = idx.cpu().numpy() if hasattr(idx, "cpu") else np.asarray(idx)
+    return {t: sparse_attn_row(f64(Qs[t]), K, V, idx[t], scale) for t in rows}
+
+
+# ---------------------------------------------------------------------------
+# Decode over the FP8 cache
+# ---------------------------------------------------------------------------
+
+def dequant_cache(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """k_j = E4M3(code_j) * scale_j, exact in fp64."""
+    return e4m3_decode(u8(codes)) * f64(scales)[:, None]
+
+
+def decode_select(Q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ks: np.ndarray,
+                  vs: np.ndarray, seqs: Sequence[int], kv_len: int, window: int,
+                  topk: int, scale: Optional[float] = None) -> Dict[int, SelectRow]:
+    """Decode: the cache of sequence b holds kv_len tokens, the new token's own
+    K/V included; its query sits at position kv_len-1 and sees keys [0, kv_len)."""
+    d = Q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = {}
+    for b in seqs:
+        K = dequant_cache(Kc[b, :kv_len], ks[b, :kv_len])
+        V = dequant_cache(Vc[b, :kv_len], vs[b, :kv_len])
+        out[b] = select_row(f64(Q[b]), K, V, kv_len - 1,
+                            window, topk, scale)
+    return out
+
+
+def sparse_attn_decode(Qs: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ks: np.ndarray,
+                       vs: np.ndarray, idx: np.ndarray, seqs: Sequence[int],
+                       scale: Optional[float] = None) -> Dict[int, np.ndarray]:
+    d = Qs.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    idx = idx.cpu().numpy() if hasattr(idx, "cpu") else np.asarray(idx)
+    out = {}
+    for b in seqs:
+        row = np.asarray(idx[b])
+        S = row[row >= 0].astype(np.int64)
+        K = dequant_cache(u8(Kc[b])[S], f64(ks[b])[S])
+        V = dequant_cache(u8(Vc[b])[S], f64(vs[b])[S])
+        local = np.arange(S.shape[0], dtype=np.int32)
+        out[b] = sparse_attn_row(f64(Qs[b]), K, V, local, scale)
+    return out
