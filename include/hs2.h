@@ -1,0 +1,188 @@
+/*
+ * hs2.h -- C ABI of libhs2.so, the B200 (sm_100a) hot path of HySparse2's
+ * token-level KV Reuse attention.
+ *
+ * Method (cited by page and passage; the pages give no code and no interface):
+ *   "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing", agihunt.info
+ *   summary, inner-level KV Reuse paragraph -- a causal full-attention layer
+ *   scores every past token; per query position the 128 most recent tokens are
+ *   forced into the selection and 1024 high-scoring out-of-window tokens are
+ *   added; the following sparse layers gather only those tokens from the same
+ *   full-attention KV.  Next paragraph: MQA (one KV head), NoPE, the full layer
+ *   acts as an oracle selector with exact attention scores.  Outer-level KV
+ *   Bridging paragraph: a cross-decoder full layer's K/V are its own linear
+ *   projections of a self-decoder full layer's hidden state.  Results table
+ *   "KV @1M (FP8)": the cache is stored in FP8.  10100.com article, "evolution
+ *   two": *at most* 1024 selected tokens.
+ *
+ * Readings fixed here where the pages are silent:
+ *   - selection score of key j for query i: sigma_ij = sum over the query heads
+ *     h of softmax_j(s_hij), s_hij = scale * q_ih . k_j (scale normally 1/sqrt(d));
+ *   - forced window of query position p = positions [p-window+1, p];
+ *     candidates = [0, p-window]; up to topk of them with the largest sigma;
+ *   - FP8 = OCP E4M3FN, round to nearest even, saturating; one fp32 scale per
+ *     token row, value = E4M3(code) * scale.
+ *
+ * Conventions common to every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned, dense row-major with the stated shape.  The library allocates
+ *     nothing; scratch comes from a caller workspace whose size the matching
+ *     *_workspace query returns.
+ *   - bf16 = IEEE bfloat16 (uint16 storage); fp8 = E4M3FN (uint8 storage).
+ *   - idx rows are int32 absolute key positions; -1 marks an empty slot.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Argument errors are reported synchronously, before any launch,
+ *     and nothing is written.  A failed launch returns HS2_ERR_CUDA.  Checks
+ *     made on the device (an idx entry out of range) and bounded waits that ran
+ *     out set a per-device status word read by hs2_device_status().
+ *   - No exception or abort crosses the ABI.  Calls on distinct workspaces may
+ *     run concurrently from several host threads.
+ *   - Supported in this version: one KV head, Hq in {8, 16}, d in {128, 256},
+ *     window + topk <= 2048, window >= 1.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HS2_API __attribute__((visibility("default")))
+#else
+#define HS2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape      */
+  HS2_ERR_UNSUPPORTED = 2,   /* valid request outside this version's shapes    */
+  HS2_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small     */
+  HS2_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed     */
+  HS2_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up              */
+  HS2_ERR_DEVICE_CHECK = 6   /* a device-side input check failed (bad idx)      */
+} hs2_status;
+
+typedef enum { HS2_KV_BF16 = 0, HS2_KV_FP8_E4M3 = 1 } hs2_kv_dtype;
+
+/* Static text for a status code. */
+HS2_API const char* hs2_status_string(hs2_status s);
+
+/* Detail of the last error on the calling host thread ("" if none). */
+HS2_API const char* hs2_last_error(void);
+
+/* Library version, e.g. "hs2 0.1 sm_100a". */
+HS2_API const char* hs2_version(void);
+
+/*
+ * KV Bridging re-projection (outer-level KV sharing; agihunt.info summary,
+ * KV Bridging paragraph).  For r < rows and c < d:
+ *     K[r,c] = sum_e hidden[r,e] * Wk[c,e],   V[r,c] = sum_e hidden[r,e] * Wv[c,e]
+ * accumulated in fp32 on the tensor cores.
+ *   hidden : bf16 [rows, hidden_dim]    (the self-decoder hidden states)
+ *   Wk, Wv : bf16 [d, hidden_dim]       (this layer's own projections, [out, in])
+ *   out_dtype HS2_KV_BF16     : K_out, V_out bf16 [rows, d], rounded to nearest even;
+ *                               k_scale, v_scale must be NULL.
+ *   out_dtype HS2_KV_FP8_E4M3 : K_out, V_out uint8 E4M3 codes [rows, d] and
+ *                               k_scale, v_scale fp32 [rows] with
+ *                               scale = amax(row)/448 (1 for an all-zero row),
+ *                               code = E4M3_RNE_satfinite(x / scale).
+ * Requires rows >= 1, hidden_dim a positive multiple of 64, d == 256.
+ */
+HS2_API hs2_status hs2_bridge_kv(const void* hidden, int64_t rows, int hidden_dim,
+                         const void* Wk, const void* Wv, int d, hs2_kv_dtype out_dtype,
+                         void* K_out, void* V_out, float* k_scale, float* v_scale,
+                         void* stream);
+
+/*
+ * Full-attention layer as the oracle selector (agihunt.info summary, KV Reuse
+ * and MQA/NoPE paragraphs).  Query t of sequence b sits at absolute position
+ * p = q_start + t and attends causally to keys 0..p of its sequence:
+ *     O[b,t,h,:] = sum_j softmax_j(scale * q . k_j) v_j
+ *     idx[b,t,0:window]            = p-window+1 .. p (-1 where negative)
+ *     idx[b,t,window:window+n]     = the n = min(topk, p-window+1) candidates
+ *                                    j <= p-window with the largest sigma_j,
+ *                                    ascending; the rest of the row is -1.
+ * Two forms are supported:
+ *   prefill: kv_dtype HS2_KV_BF16, batch == 1, Tq >= 1, q_start + Tq <= kv_len.
+ *            Q bf16 [Tq, Hq, d]; K, V bf16 [kv_len, d]; k_scale/v_scale NULL.
+ *            A long prefill may be issued in query chunks (q_start > 0) over
+ *            the causal prefix (kv_len = q_start + Tq).
+ *   decode : kv_dtype HS2_KV_FP8_E4M3, batch >= 1, Tq == 1,
+ *            q_start == kv_len - 1 (the cache already holds the new token).
+ *            Q bf16 [batch, Hq, d]; K, V uint8 [batch, kv_stride_tokens, d];
+ *            k_scale, v_scale fp32 [batch, kv_stride_tokens]; key j of
+ *            sequence b is E4M3(K[b,j,:]) * k_scale[b,j] (V likewise).
+ * kv_stride_tokens >= kv_len (prefill: ignored, rows are contiguous).
+ * Outputs: O bf16 [batch, Tq, Hq, d]; idx int32 [batch, Tq, window+topk].
+ * workspace: device memory of at least hs2_full_attn_select_workspace() bytes,
+ * 256-byte aligned; its contents on entry do not matter.
+ */
+HS2_API hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V,
+                                const float* k_scale, const float* v_scale,
+                                hs2_kv_dtype kv_dtype, int batch, int64_t q_start,
+                                int64_t Tq, int64_t kv_len, int64_t kv_stride_tokens,
+                                int Hq, int d, int window, int topk, float softmax_scale,
+                                void* O, int32_t* idx, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* Workspace bytes hs2_full_attn_select needs for these shape arguments. */
+HS2_API hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int64_t Tq,
+                                          int64_t kv_len, int Hq, int d, int window,
+                                          int topk, size_t* bytes);
+
+/*
+ * Sparse layer, prefill (agihunt.info summary, KV Reuse paragraph: the sparse
+ * layers reuse the selected tokens of the full layer's KV).  For each query t:
+ *     O[t,h,:] = sum_{j in S_t} softmax_{S_t}(scale * q_th . k_j) v_j,
+ *     S_t = { idx[t,s] : idx[t,s] >= 0 }.
+ *   Q bf16 [Tq, Hq, d] (this sparse layer's own queries); K, V bf16 [kv_len, d]
+ *   (the full layer's KV); idx int32 [Tq, n_idx]; O bf16 [Tq, Hq, d].
+ * An entry idx >= kv_len (or < -1) is skipped and raises HS2_ERR_DEVICE_CHECK
+ * in hs2_device_status(); a row with no valid entry yields O = 0.
+ */
+HS2_API hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V,
+                                   const int32_t* idx, int64_t Tq, int64_t kv_len, int n_idx,
+                                   int Hq, int d, float softmax_scale, void* O, void* stream);
+
+/*
+ * Sparse layer, decode over the FP8 cache: as hs2_sparse_attn_prefill with one
+ * query per sequence, keys dequantised as E4M3(code) * scale.
+ *   Q bf16 [batch, Hq, d]; Kc, Vc uint8 [batch, kv_stride_tokens, d];
+ *   k_scale, v_scale fp32 [batch, kv_stride_tokens]; idx int32 [batch, n_idx]
+ *   with entries < kv_len; O bf16 [batch, Hq, d].
+ * kv_dtype must be HS2_KV_FP8_E4M3.  workspace may be NULL when
+ * hs2_sparse_attn_decode_workspace() returns 0.
+ */
+HS2_API hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
+                                  const float* k_scale, const float* v_scale,
+                                  hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                                  int64_t kv_stride_tokens, const int32_t* idx, int n_idx,
+                                  int Hq, int d, float softmax_scale, void* O,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+HS2_API hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d,
+                                            size_t* bytes);
+
+/*
+ * Synchronises `stream`, then reads and clears the status word of the current
+ * device: HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA if
+ * the synchronisation itself failed).
+ */
+HS2_API hs2_status hs2_device_status(void* stream);
+
+/*
+ * Test hook for the bounded device waits: sets the iteration limit of every
+ * inter-CTA spin-wait the library launches afterwards on the current device
+ * (0 restores the default).  A limit of 1 makes a wait that is not already
+ * satisfied give up at once and report HS2_ERR_TIMEOUT.
+ */
+HS2_API hs2_status hs2_set_spin_limit(int64_t iterations);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HS2_H_ */

@@ -1,0 +1,210 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Sizes the oracle finishes in seconds that still span several tiles and a
+ragged tail; edge cases (rows with fewer candidates than top-k, fewer keys
+than the window, a single query, chunked prefill, invalid idx entries, the
+bounded-wait timeout path)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from hs2_cases import (bf16_rule, check_select_rows, fp8_rule, gpu_decode_select, gpu_prefill_select,
+                       gpu_sparse_decode, gpu_sparse_prefill)
+from parity import TOL_BF16, TOL_FP8, check_idx_row, max_abs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hs2():
+    import token_level_kv_b200 as m
+    return m
+
+
+# ---------------------------------------------------------------- bridging
+
+@pytest.mark.parametrize("rows,D", [(333, 2048), (128, 512), (1, 64)])
+def test_bridge_bf16(hs2, rows, D):
+    c = synth.make_bridge_case(rows, D, 256, 1, seed=1)
+    h, Wk, Wv = c.hidden.cuda(), c.Wk[0].cuda(), c.Wv[0].cuda()
+    K = torch.empty(rows, 256, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    hs2.hs2_bridge_kv(h, Wk, Wv, K, V)
+    assert hs2.hs2_device_status() == 0
+    for got, W in ((K, c.Wk[0]), (V, c.Wv[0])):
+        exact = oracle.bridge_rows(c.hidden, W)
+        bad, err = bf16_rule(got.cpu(), exact)
+        assert bad == 0, f"{bad} bf16 outputs off by more than the rounding rule (max err {err})"
+
+
+@pytest.mark.parametrize("rows", [333, 1000])
+def test_bridge_fp8(hs2, rows):
+    c = synth.make_bridge_case(rows, 2048, 256, 1, seed=2)
+    c.hidden[5] = 0          # an all-zero hidden row -> all-zero K/V row, scale 1
+    h, Wk, Wv = c.hidden.cuda(), c.Wk[0].cuda(), c.Wv[0].cuda()
+    K = torch.empty(rows, 256, dtype=torch.uint8, device="cuda")
+    V = torch.empty_like(K)
+    ks = torch.empty(rows, dtype=torch.float32, device="cuda")
+    vs = torch.empty_like(ks)
+    hs2.hs2_bridge_kv(h, Wk, Wv, K, V, ks, vs)
+    assert hs2.hs2_device_status() == 0
+    for codes, sc, W in ((K, ks, c.Wk[0]), (V, vs, c.Wv[0])):
+        exact = oracle.bridge_rows(c.hidden, W)
+        assert float(sc[5]) == 1.0 and int(codes[5].abs().sum()) == 0
+        nz = np.abs(exact).max(1) > 0
+        srel, bad = fp8_rule(codes.cpu()[nz], sc.cpu()[nz], exact[nz])
+        assert srel <= 1e-5, f"scale relative error {srel}"
+        assert bad == 0, f"{bad} FP8 codes off by more than the rounding rule"
+
+
+# ---------------------------------------------------------------- prefill select
+
+def test_prefill_select_small_h8_d128(hs2):
+    """1024 queries, 8 heads, d = 128, window 128 + top-256, 4 needles: all rows."""
+    c = synth.CONFIGS[1]
+    case = synth.make_prefill_case(c["T"], c["H"], c["d"], c["window"], c["topk"], n_sparse=1,
+                                   n_needles=c["n_needles"], seed=0)
+    O, idx = gpu_prefill_select(case)
+    ref, worst, swaps = check_select_rows(case, O, idx, range(case.T))
+    for p, i in case.needles:
+        assert p in set(idx[i, case.window:].tolist())
+    # sparse layer on the oracle's index set (identical inputs on both sides)
+    oidx = np.stack([ref[t].idx for t in range(case.T)])
+    Os = gpu_sparse_prefill(case.Q_sparse[0], case.K, case.V, oidx)
+    sref = oracle.sparse_attn(case.Q_sparse[0], case.K, case.V, oidx, range(case.T))
+    assert max(max_abs(Os[t].float().numpy(), sref[t]) for t in range(case.T)) <= TOL_BF16
+    # end to end on the GPU's own index set where it equals the oracle's
+    Os2 = gpu_sparse_prefill(case.Q_sparse[0], case.K, case.V, idx.numpy())
+    same = [t for t in range(case.T) if np.array_equal(idx[t].numpy(), oidx[t])]
+    assert len(same) >= case.T // 2
+    assert max(max_abs(Os2[t].float().numpy(), sref[t]) for t in same) <= TOL_BF16
+
+
+@pytest.mark.parametrize("T", [1500, 200, 1])
+def test_prefill_select_h16_d256(hs2, T):
+    """16 heads, d = 256, window 128 + top-1024: rows with fewer candidates
+    than top-k, fewer keys than the window, a ragged last query tile."""
+    case = synth.make_prefill_case(T, 16, 256, 128, 1024, n_sparse=1, n_needles=2 if T > 300 else 0,
+                                   seed=4)
+    O, idx = gpu_prefill_select(case)
+    rows = range(T)
+    check_select_rows(case, O, idx, rows)
+
+
+def test_prefill_select_scaled_inputs_tie_margin(hs2):
+    """N(0,1)/16 inputs: near-uniform attention, selection decided by tiny gaps."""
+    case = synth.make_prefill_case(2600, 16, 256, 128, 1024, n_sparse=0, n_needles=8, scale=1 / 16, seed=5)
+    O, idx = gpu_prefill_select(case)
+    rows = list(range(1100, 1200)) + list(range(2500, 2600)) + [i for _, i in case.needles]
+    _, _, swaps = check_select_rows(case, O, idx, rows)
+    for p, i in case.needles:
+        assert p in set(idx[i, case.window:].tolist())
+
+
+def test_chunked_prefill_equals_one_call(hs2):
+    """Query chunks over the causal prefix give the same rows, bit for bit."""
+    case = synth.make_prefill_case(1800, 16, 256, 128, 1024, n_sparse=0, seed=6)
+    O1, idx1 = gpu_prefill_select(case)
+    Oa, idxa = gpu_prefill_select(case, q_start=0, Tq=904)
+    Ob, idxb = gpu_prefill_select(case, q_start=904, Tq=896)
+    assert torch.equal(torch.cat([idxa, idxb]), idx1)
+    assert torch.equal(torch.cat([Oa, Ob]), O1)
+    check_select_rows(case, Ob, idxb, [0, 1, 500, 895], q_start=904)
+
+
+# ---------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("B,N", [(3, 5000), (2, 1200), (1, 100), (2, 4097)])
+def test_decode_select_fp8(hs2, B, N):
+    case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=1, seed=7)
+    O, idx = gpu_decode_select(case)
+    ref = oracle.decode_select(case.Q, case.Kc, case.Vc, case.ks, case.vs, range(B), N, 128, 1024)
+    for b in range(B):
+        ok, _, msg = check_idx_row(idx[b].numpy(), ref[b], 128, 1024)
+        assert ok, msg
+        assert max_abs(O[b].float().numpy(), ref[b].O) <= TOL_FP8
+    oidx = np.stack([ref[b].idx for b in range(B)])
+    Os = gpu_sparse_decode(case, case.Q_sparse[0], oidx)
+    sref = oracle.sparse_attn_decode(case.Q_sparse[0], case.Kc, case.Vc, case.ks, case.vs, oidx, range(B))
+    for b in range(B):
+        assert max_abs(Os[b].float().numpy(), sref[b]) <= TOL_FP8
+
+
+def test_sparse_decode_many_sequences(hs2):
+    """More sequences than SMs' worth of splits, kv_len below the row stride."""
+    B, N = 70, 3000
+    case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=1, seed=8)
+    g = np.random.default_rng(0)
+    idx = np.full((B, 1152), -1, dtype=np.int32)
+    for b in range(B):
+        n = int(g.integers(1, 1153))
+        idx[b, :n] = np.sort(g.choice(2900, size=n, replace=False))
+    O = gpu_sparse_decode(case, case.Q_sparse[0], idx, kv_len=2900)
+    ref = oracle.sparse_attn_decode(case.Q_sparse[0], case.Kc, case.Vc, case.ks, case.vs, idx, range(B))
+    assert max(max_abs(O[b].float().numpy(), ref[b]) for b in range(B)) <= TOL_FP8
+
+
+# ---------------------------------------------------------------- checks and faults
+
+def test_sparse_prefill_bad_index_is_reported_and_skipped(hs2):
+    T, H, d = 40, 16, 128
+    case = synth.make_prefill_case(T, H, d, 8, 8, n_sparse=1, seed=9)
+    idx = np.full((T, 16), -1, dtype=np.int32)
+    for t in range(T):
+        idx[t, :t + 1 if t < 16 else 16] = np.arange(min(t + 1, 16))
+    bad = idx.copy()
+    bad[3, 1] = 10 ** 6                       # outside the KV
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device="cuda")
+    hs2.hs2_sparse_attn_prefill(case.Q_sparse[0].cuda(), case.K.cuda(), case.V.cuda(),
+                                torch.from_numpy(bad).cuda(), O)
+    assert hs2.hs2_device_status() == 6      # HS2_ERR_DEVICE_CHECK
+    assert hs2.hs2_device_status() == 0      # the word is cleared once read
+    skipped = idx.copy()
+    skipped[3, 1] = -1
+    ref = oracle.sparse_attn(case.Q_sparse[0], case.K, case.V, skipped, range(T))
+    assert max(max_abs(O[t].float().cpu().numpy(), ref[t]) for t in range(T)) <= TOL_BF16
+
+
+def test_argument_errors_do_not_launch(hs2):
+    K = torch.empty(10, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_bridge_kv(torch.empty(10, 100, dtype=torch.bfloat16, device="cuda"),
+                          torch.empty(256, 100, dtype=torch.bfloat16, device="cuda"),
+                          torch.empty(256, 100, dtype=torch.bfloat16, device="cuda"), K, K)
+    assert e.value.status == 1
+    Q = torch.empty(4, 16, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_full_attn_select(Q, K, K, Q, torch.empty(4, 1152, dtype=torch.int32, device="cuda"),
+                                 torch.empty(64, dtype=torch.uint8, device="cuda"), window=128, topk=1024)
+    assert e.value.status == 3               # workspace too small
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_full_attn_select(torch.empty(4, 12, 256, dtype=torch.bfloat16, device="cuda"), K, K, Q,
+                                 torch.empty(4, 1152, dtype=torch.int32, device="cuda"),
+                                 torch.empty(1 << 20, dtype=torch.uint8, device="cuda"), window=128, topk=1024)
+    assert e.value.status == 2               # 12 heads: unsupported
+    assert hs2.hs2_device_status() == 0
+
+
+def test_bounded_wait_gives_up_and_context_survives(hs2):
+    """With a wait limit of one try the tensor-core kernel's waits give up: the
+    call reports HS2_ERR_TIMEOUT through the status word, the CTAs drain their
+    own copies and MMAs, and the next call with the default limit is exact."""
+    c = synth.make_bridge_case(4096, 2048, 256, 1, seed=3)
+    h, Wk, Wv = c.hidden.cuda(), c.Wk[0].cuda(), c.Wv[0].cuda()
+    K = torch.empty(4096, 256, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    hs2.hs2_set_spin_limit(1)
+    try:
+        hs2.hs2_bridge_kv(h, Wk, Wv, K, V)
+        st = hs2.hs2_device_status()
+    finally:
+        hs2.hs2_set_spin_limit(0)
+    assert st == 5                           # HS2_ERR_TIMEOUT
+    hs2.hs2_bridge_kv(h, Wk, Wv, K, V)
+    assert hs2.hs2_device_status() == 0
+    bad, _ = bf16_rule(K[:300].cpu(), oracle.bridge_rows(c.hidden[:300], c.Wk[0]))
+    assert bad == 0

@@ -1,0 +1,187 @@
+"""Python binding of libhs2.so -- the HySparse2 token-level KV Reuse hot path
+on B200 (sm_100a).
+
+Argument marshalling only: shapes are read off the tensors, pointers and the
+current CUDA stream are passed to the C ABI (include/hs2.h), and a non-zero
+status is raised as Hs2Error.  Every step of the computation runs in the
+library's CUDA kernels; there is no other code path.  PyTorch is used for
+device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhs2.so")
+
+KV_BF16 = 0
+KV_FP8_E4M3 = 1
+
+STATUS = {0: "HS2_OK", 1: "HS2_ERR_INVALID_ARG", 2: "HS2_ERR_UNSUPPORTED", 3: "HS2_ERR_WORKSPACE",
+          4: "HS2_ERR_CUDA", 5: "HS2_ERR_TIMEOUT", 6: "HS2_ERR_DEVICE_CHECK"}
+
+
+class Hs2Error(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m token_level_kv_b200.build` "
+                          "(nvcc, sm_100a); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, L, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "hs2_status_string": ([I], ctypes.c_char_p),
+        "hs2_last_error": ([], ctypes.c_char_p),
+        "hs2_version": ([], ctypes.c_char_p),
+        "hs2_bridge_kv": ([P, L, I, P, P, I, I, P, P, P, P, P], I),
+        "hs2_full_attn_select": ([P, P, P, P, P, I, I, L, L, L, L, I, I, I, I, F, P, P, P, Z, P], I),
+        "hs2_full_attn_select_workspace": ([I, I, L, L, I, I, I, I, ctypes.POINTER(Z)], I),
+        "hs2_sparse_attn_prefill": ([P, P, P, P, L, L, I, I, I, F, P, P], I),
+        "hs2_sparse_attn_decode": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P, Z, P], I),
+        "hs2_sparse_attn_decode_workspace": ([I, I, I, I, ctypes.POINTER(Z)], I),
+        "hs2_device_status": ([P], I),
+        "hs2_set_spin_limit": ([L], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+lib = _load()
+EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv", "hs2_full_attn_select",
+           "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
+           "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit")
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise Hs2Error(status, lib.hs2_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("hs2 takes device tensors only (got a CPU tensor)")
+    if not t.is_contiguous():
+        raise ValueError("hs2 takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _kv_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KV_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return KV_FP8_E4M3
+    raise ValueError(f"K/V must be bf16 or FP8 E4M3 codes, got {t.dtype}")
+
+
+def hs2_version() -> str:
+    return lib.hs2_version().decode()
+
+
+def hs2_bridge_kv(hidden, Wk, Wv, K_out, V_out, k_scale=None, v_scale=None, stream=None) -> None:
+    """K_out = hidden Wk^T, V_out = hidden Wv^T; FP8 codes + row scales when K_out is uint8."""
+    rows, D = hidden.shape
+    d = Wk.shape[0]
+    out = _kv_dtype(K_out)
+    _check(lib.hs2_bridge_kv(_ptr(hidden), rows, D, _ptr(Wk), _ptr(Wv), d, out, _ptr(K_out), _ptr(V_out),
+                             _ptr(k_scale), _ptr(v_scale), _stream(stream)))
+
+
+def hs2_full_attn_select_workspace(kv_dtype: int, batch: int, Tq: int, kv_len: int, Hq: int, d: int,
+                                   window: int, topk: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hs2_full_attn_select_workspace(kv_dtype, batch, Tq, kv_len, Hq, d, window, topk, ctypes.byref(n)))
+    return n.value
+
+
+def hs2_full_attn_select(Q, K, V, O, idx, workspace, *, window: int, topk: int, q_start: int = 0,
+                         kv_len: int | None = None, k_scale=None, v_scale=None,
+                         softmax_scale: float | None = None, stream=None) -> None:
+    """Full-attention layer + token selection.
+
+    prefill (bf16 K/V): Q [Tq, H, d], K/V [>= kv_len, d], O [Tq, H, d], idx [Tq, window+topk].
+    decode (FP8 K/V codes): Q [B, H, d], K/V [B, stride, d], k/v_scale [B, stride],
+    O [B, H, d], idx [B, window+topk]; the query sits at kv_len - 1.
+    """
+    kvd = _kv_dtype(K)
+    d = Q.shape[-1]
+    H = Q.shape[-2]
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    if kvd == KV_BF16:
+        batch, Tq = 1, Q.shape[0]
+        kv_len = K.shape[0] if kv_len is None else kv_len
+        stride = kv_len
+    else:
+        batch, Tq = Q.shape[0], 1
+        stride = K.shape[1]
+        kv_len = stride if kv_len is None else kv_len
+        q_start = kv_len - 1
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.hs2_full_attn_select(_ptr(Q), _ptr(K), _ptr(V), _ptr(k_scale), _ptr(v_scale), kvd, batch,
+                                    q_start, Tq, kv_len, stride, H, d, window, topk, scale, _ptr(O), _ptr(idx),
+                                    _ptr(workspace), ws, _stream(stream)))
+
+
+def hs2_sparse_attn_prefill(Q, K, V, idx, O, *, kv_len: int | None = None, softmax_scale: float | None = None,
+                            stream=None) -> None:
+    """Sparse layer: Q [Tq, H, d] over the rows idx [Tq, n_idx] of the shared K/V [kv_len, d]."""
+    Tq, H, d = Q.shape
+    kv_len = K.shape[0] if kv_len is None else kv_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    _check(lib.hs2_sparse_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), Tq, kv_len, idx.shape[-1], H, d,
+                                       scale, _ptr(O), _stream(stream)))
+
+
+def hs2_sparse_attn_decode_workspace(batch: int, n_idx: int, Hq: int, d: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, ctypes.byref(n)))
+    return n.value
+
+
+def hs2_sparse_attn_decode(Q, Kc, Vc, k_scale, v_scale, idx, O, workspace=None, *, kv_len: int | None = None,
+                           softmax_scale: float | None = None, stream=None) -> None:
+    """Sparse layer over the FP8 cache: Q [B, H, d], Kc/Vc [B, stride, d] codes, idx [B, n_idx]."""
+    B, H, d = Q.shape
+    stride = Kc.shape[1]
+    kv_len = stride if kv_len is None else kv_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.hs2_sparse_attn_decode(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale), KV_FP8_E4M3, B,
+                                      kv_len, stride, _ptr(idx), idx.shape[-1], H, d, scale, _ptr(O),
+                                      _ptr(workspace), ws, _stream(stream)))
+
+
+def hs2_device_status(stream=None) -> int:
+    """Synchronises the stream; returns the device status (0 = OK) and clears it."""
+    return lib.hs2_device_status(_stream(stream))
+
+
+def hs2_set_spin_limit(iterations: int) -> None:
+    _check(lib.hs2_set_spin_limit(iterations))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor | None:
+    """A 256-byte aligned device buffer of at least nbytes (None for 0)."""
+    if nbytes == 0:
+        return None
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,554 @@
+// libhs2.so: the C ABI declared in include/hs2.h.  Argument checks, workspace
+// sizing, TMA tensor maps and kernel launches; all compute is in the kernels
+// included below (one translation unit).
+#include "hs2.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn16.cuh"
+#include "bridge_gemm.cuh"
+#include "common.cuh"
+#include "fa_fwd.cuh"
+#include "select_sigma.cuh"
+#include "topk.cuh"
+
+namespace hs2 {
+
+__device__ unsigned g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kDefaultSpin = 1ll << 40;   // the 4 s time cap bounds it
+thread_local char g_err[512] = "";
+long long g_spin[kMaxDevices];
+unsigned* g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+std::mutex g_mu;
+
+hs2_status fail(hs2_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define HS2_CHECK(cond, status, ...)        \
+  do {                                      \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+hs2_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(HS2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Per-device state: status-word address, SM count, spin limit.
+hs2_status device_ctx(DevCtx* ctx, int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HS2_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) return fail(HS2_ERR_UNSUPPORTED, "libhs2 is built for sm_100a (compute capability 10.x), device has %d.x", major);
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+    g_num_sms[dev] = sms;
+  }
+  ctx->status = g_status_ptr[dev];
+  ctx->spin_limit = g_spin[dev] > 0 ? g_spin[dev] : kDefaultSpin;
+  if (num_sms) *num_sms = g_num_sms[dev];
+  return HS2_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (row stride in elements), 128-byte swizzle.
+hs2_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
+                         uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {stride_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HS2_OK;
+}
+
+hs2_status after_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return HS2_OK;
+}
+
+template <typename K>
+hs2_status set_smem(K kernel, size_t bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return HS2_OK;
+}
+
+bool shape_ok(int Hq, int d) { return (Hq == 8 || Hq == 16) && (d == 128 || d == 256); }
+
+// ------------------------------------------------------------------ workspace
+struct PrefillWs {
+  size_t ml, sigma, total;
+  int64_t ld;
+};
+PrefillWs prefill_ws(int64_t Tq, int64_t kv_len, int Hq) {
+  PrefillWs w;
+  w.ld = round_up(kv_len, 64);
+  w.ml = up256((size_t)Tq * Hq * 2 * sizeof(float));
+  w.sigma = up256((size_t)Tq * (size_t)w.ld * sizeof(float));
+  w.total = w.ml + w.sigma;
+  return w;
+}
+
+constexpr int kDecodeKeysPerSplit = 2048;
+struct DecodeWs {
+  size_t logits, part, ml, sigma, total;
+  int64_t ld;
+  int splits;
+};
+DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d) {
+  DecodeWs w;
+  w.ld = round_up(kv_len, 64);
+  w.splits = (int)((kv_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit);
+  w.logits = up256((size_t)batch * Hq * (size_t)w.ld * sizeof(float));
+  w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
+  w.ml = up256((size_t)batch * Hq * 2 * sizeof(float));
+  w.sigma = up256((size_t)batch * (size_t)w.ld * sizeof(float));
+  w.total = w.logits + w.part + w.ml + w.sigma;
+  return w;
+}
+
+int sparse_decode_splits(int batch, int n_idx, int num_sms) {
+  int s = (num_sms + batch - 1) / batch;
+  const int max_s = std::max(1, (n_idx + 63) / 64);
+  return std::max(1, std::min(s, max_s));
+}
+
+// ------------------------------------------------------------------ launches
+template <int D, bool FP8, bool RANGE>
+hs2_status launch_attn16(const Attn16Params& p, int grid, cudaStream_t st, const DevCtx& ctx) {
+  constexpr size_t smem = A16Layout<D, FP8>::SMEM;
+  hs2_status s = set_smem(attn16_kernel<D, FP8, RANGE>, smem);
+  if (s != HS2_OK) return s;
+  attn16_kernel<D, FP8, RANGE><<<grid, 128, smem, st>>>(p, ctx);
+  return after_launch("attn16_kernel");
+}
+
+template <int D>
+hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
+                          cudaStream_t st) {
+  attn16_combine_kernel<D><<<items, 256, 0, st>>>(part, splits, H, O, ml);
+  return after_launch("attn16_combine_kernel");
+}
+
+template <int D>
+hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q_start, int64_t Tq, int64_t kv_len,
+                          int Hq, int window, int topk, float scale, void* O, int32_t* idx, void* ws,
+                          cudaStream_t st, const DevCtx& ctx) {
+  const PrefillWs w = prefill_ws(Tq, kv_len, Hq);
+  float* ml = reinterpret_cast<float*>(ws);
+  float* sigma = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.ml);
+  const float sl2 = scale * 1.4426950408889634f;
+  CUtensorMap mQ, mQ256, mK, mV;
+  hs2_status s;
+  if ((s = make_map_bf16(&mQ, Q, D, (uint64_t)Tq * Hq, D, 64, 128)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mQ256, Q, D, (uint64_t)Tq * Hq, D, 64, 256)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mK, K, D, (uint64_t)kv_len, D, 64, 128)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mV, V, D, (uint64_t)kv_len, D, 64, 128)) != HS2_OK) return s;
+
+  FaParams fp;
+  fp.Tq = Tq;
+  fp.q_start = q_start;
+  fp.kv_len = kv_len;
+  fp.H = Hq;
+  fp.scale_log2 = sl2;
+  fp.O = static_cast<__nv_bfloat16*>(O);
+  fp.ml = ml;
+  fp.n_qtiles = (int)((Tq * Hq + 127) / 128);
+  if ((s = set_smem(fa_fwd_kernel<D>, FaLayout<D>::SMEM)) != HS2_OK) return s;
+  fa_fwd_kernel<D><<<fp.n_qtiles, FA_THREADS, FaLayout<D>::SMEM, st>>>(mQ, mK, mV, fp, ctx);
+  if ((s = after_launch("fa_fwd_kernel")) != HS2_OK) return s;
+
+  SgParams sp;
+  sp.Tq = Tq;
+  sp.q_start = q_start;
+  sp.kv_len = kv_len;
+  sp.H = Hq;
+  sp.window = window;
+  sp.scale_log2 = sl2;
+  sp.ml = ml;
+  sp.sigma = sigma;
+  sp.ld = w.ld;
+  sp.n_groups = (int)((Tq * Hq + 255) / 256);
+  if (Hq == 16) {
+    if ((s = set_smem(select_sigma_kernel<D, 16>, SgLayout<D>::SMEM)) != HS2_OK) return s;
+    select_sigma_kernel<D, 16><<<sp.n_groups, SG_THREADS, SgLayout<D>::SMEM, st>>>(mQ256, mK, sp, ctx);
+  } else {
+    if ((s = set_smem(select_sigma_kernel<D, 8>, SgLayout<D>::SMEM)) != HS2_OK) return s;
+    select_sigma_kernel<D, 8><<<sp.n_groups, SG_THREADS, SgLayout<D>::SMEM, st>>>(mQ256, mK, sp, ctx);
+  }
+  if ((s = after_launch("select_sigma_kernel")) != HS2_OK) return s;
+
+  TopkParams tp;
+  tp.sigma = sigma;
+  tp.ld = w.ld;
+  tp.p0 = q_start;
+  tp.pstep = 1;
+  tp.window = window;
+  tp.topk = topk;
+  tp.idx = idx;
+  if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
+  topk_select_kernel<<<(unsigned)Tq, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
+  return after_launch("topk_select_kernel");
+}
+
+template <int D>
+hs2_status decode_select(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
+                         int64_t kv_len, int64_t kv_stride, int Hq, int window, int topk, float scale, void* O,
+                         int32_t* idx, void* ws, cudaStream_t st, const DevCtx& ctx) {
+  const DecodeWs w = decode_ws(batch, kv_len, Hq, D);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  float* logits = reinterpret_cast<float*>(b);
+  float* part = reinterpret_cast<float*>(b + w.logits);
+  float* ml = reinterpret_cast<float*>(b + w.logits + w.part);
+  float* sigma = reinterpret_cast<float*>(b + w.logits + w.part + w.ml);
+  Attn16Params p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = K;
+  p.V = V;
+  p.ks = ks;
+  p.vs = vs;
+  p.idx = nullptr;
+  p.n_idx = 0;
+  p.kv_len = kv_len;
+  p.kv_stride = kv_stride;
+  p.H = Hq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.splits = w.splits;
+  p.slots_per_split = kDecodeKeysPerSplit;
+  p.final_out = 0;
+  p.O = nullptr;
+  p.part = part;
+  p.logits = logits;
+  p.logit_ld = w.ld;
+  hs2_status s = launch_attn16<D, true, true>(p, batch * w.splits, st, ctx);
+  if (s != HS2_OK) return s;
+  if ((s = launch_combine<D>(part, w.splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
+  const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
+  if (n_cand > 0) {
+    dim3 g((unsigned)((n_cand + 255) / 256), (unsigned)batch);
+    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld);
+    if ((s = after_launch("decode_sigma_kernel")) != HS2_OK) return s;
+  }
+  TopkParams tp;
+  tp.sigma = sigma;
+  tp.ld = w.ld;
+  tp.p0 = kv_len - 1;
+  tp.pstep = 0;
+  tp.window = window;
+  tp.topk = topk;
+  tp.idx = idx;
+  if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
+  topk_select_kernel<<<(unsigned)batch, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
+  return after_launch("topk_select_kernel");
+}
+
+}  // namespace
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+const char* hs2_status_string(hs2_status s) {
+  switch (s) {
+    case HS2_OK: return "HS2_OK";
+    case HS2_ERR_INVALID_ARG: return "HS2_ERR_INVALID_ARG";
+    case HS2_ERR_UNSUPPORTED: return "HS2_ERR_UNSUPPORTED";
+    case HS2_ERR_WORKSPACE: return "HS2_ERR_WORKSPACE";
+    case HS2_ERR_CUDA: return "HS2_ERR_CUDA";
+    case HS2_ERR_TIMEOUT: return "HS2_ERR_TIMEOUT";
+    case HS2_ERR_DEVICE_CHECK: return "HS2_ERR_DEVICE_CHECK";
+  }
+  return "unknown hs2_status";
+}
+
+const char* hs2_last_error(void) { return g_err; }
+
+const char* hs2_version(void) { return "hs2 0.1 sm_100a"; }
+
+hs2_status hs2_bridge_kv(const void* hidden, int64_t rows, int hidden_dim, const void* Wk, const void* Wv, int d,
+                         hs2_kv_dtype out_dtype, void* K_out, void* V_out, float* k_scale, float* v_scale,
+                         void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(hidden && Wk && Wv && K_out && V_out, HS2_ERR_INVALID_ARG, "null tensor pointer");
+  HS2_CHECK(aligned16(hidden) && aligned16(Wk) && aligned16(Wv) && aligned16(K_out) && aligned16(V_out),
+            HS2_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  HS2_CHECK(rows >= 1 && rows < (1ll << 31), HS2_ERR_INVALID_ARG, "rows = %lld out of range", (long long)rows);
+  HS2_CHECK(hidden_dim > 0 && hidden_dim % 64 == 0, HS2_ERR_INVALID_ARG, "hidden_dim must be a positive multiple of 64");
+  HS2_CHECK(out_dtype == HS2_KV_BF16 || out_dtype == HS2_KV_FP8_E4M3, HS2_ERR_INVALID_ARG, "bad out_dtype");
+  HS2_CHECK(d == 256, HS2_ERR_UNSUPPORTED, "bridging supports d == 256 (got %d)", d);
+  if (out_dtype == HS2_KV_FP8_E4M3) {
+    HS2_CHECK(k_scale && v_scale && aligned4(k_scale) && aligned4(v_scale), HS2_ERR_INVALID_ARG,
+              "FP8 output needs 4-byte aligned k_scale and v_scale");
+  } else {
+    HS2_CHECK(!k_scale && !v_scale, HS2_ERR_INVALID_ARG, "bf16 output takes no scales");
+  }
+  DevCtx ctx;
+  int sms = 0;
+  hs2_status s = device_ctx(&ctx, &sms);
+  if (s != HS2_OK) return s;
+  CUtensorMap mA, mWk, mWv;
+  if ((s = make_map_bf16(&mA, hidden, hidden_dim, rows, hidden_dim, 64, 128)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mWk, Wk, hidden_dim, 256, hidden_dim, 64, 256)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mWv, Wv, hidden_dim, 256, hidden_dim, 64, 256)) != HS2_OK) return s;
+  BridgeParams p;
+  p.rows = rows;
+  p.kdim = hidden_dim;
+  p.out_fp8 = out_dtype == HS2_KV_FP8_E4M3;
+  p.K_out = K_out;
+  p.V_out = V_out;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.num_tiles = (int)(2 * ((rows + BG_BM - 1) / BG_BM));
+  if ((s = set_smem(bridge_gemm_kernel, BG_SMEM)) != HS2_OK) return s;
+  const int grid = std::min(p.num_tiles, sms);
+  bridge_gemm_kernel<<<grid, BG_THREADS, BG_SMEM, static_cast<cudaStream_t>(stream)>>>(mA, mWk, mWv, p, ctx);
+  return after_launch("bridge_gemm_kernel");
+}
+
+hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int64_t Tq, int64_t kv_len, int Hq,
+                                          int d, int window, int topk, size_t* bytes) {
+  g_err[0] = 0;
+  HS2_CHECK(bytes, HS2_ERR_INVALID_ARG, "bytes is null");
+  HS2_CHECK(batch >= 1 && Tq >= 1 && kv_len >= 1 && window >= 1 && topk >= 1, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  if (kv_dtype == HS2_KV_BF16) {
+    *bytes = prefill_ws(Tq, kv_len, Hq).total;
+  } else if (kv_dtype == HS2_KV_FP8_E4M3) {
+    *bytes = decode_ws(batch, kv_len, Hq, d).total;
+  } else {
+    return fail(HS2_ERR_INVALID_ARG, "bad kv_dtype");
+  }
+  return HS2_OK;
+}
+
+hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V, const float* k_scale,
+                                const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t q_start, int64_t Tq,
+                                int64_t kv_len, int64_t kv_stride_tokens, int Hq, int d, int window, int topk,
+                                float softmax_scale, void* O, int32_t* idx, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(Q && K && V && O && idx, HS2_ERR_INVALID_ARG, "null tensor pointer");
+  HS2_CHECK(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned16(idx), HS2_ERR_INVALID_ARG,
+            "tensor pointers must be 16-byte aligned");
+  HS2_CHECK(batch >= 1 && Tq >= 1 && kv_len >= 1 && q_start >= 0, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(window >= 1 && topk >= 1, HS2_ERR_INVALID_ARG, "window and topk must be >= 1");
+  HS2_CHECK(window + topk <= 2048, HS2_ERR_UNSUPPORTED, "window + topk must be <= 2048");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256 (got %d, %d)", Hq, d);
+  HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  HS2_CHECK(kv_len - window <= (1ll << 20), HS2_ERR_UNSUPPORTED, "at most 2^20 candidate keys per query");
+  HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0), HS2_ERR_WORKSPACE,
+            "workspace must be non-null and 256-byte aligned");
+  size_t need = 0;
+  hs2_status s = hs2_full_attn_select_workspace(kv_dtype, batch, Tq, kv_len, Hq, d, window, topk, &need);
+  if (s != HS2_OK) return s;
+  HS2_CHECK(ws_bytes >= need, HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  DevCtx ctx;
+  if ((s = device_ctx(&ctx, nullptr)) != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kv_dtype == HS2_KV_BF16) {
+    HS2_CHECK(batch == 1, HS2_ERR_UNSUPPORTED, "bf16 prefill takes batch == 1");
+    HS2_CHECK(!k_scale && !v_scale, HS2_ERR_INVALID_ARG, "bf16 KV takes no scales");
+    HS2_CHECK(q_start + Tq <= kv_len, HS2_ERR_INVALID_ARG, "q_start + Tq must be <= kv_len");
+    HS2_CHECK(Tq * Hq < (1ll << 31) && kv_len < (1ll << 31), HS2_ERR_UNSUPPORTED, "sizes beyond int32 tiles");
+    return d == 256 ? prefill_select<256>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, softmax_scale, O, idx,
+                                          workspace, st, ctx)
+                    : prefill_select<128>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, softmax_scale, O, idx,
+                                          workspace, st, ctx);
+  }
+  HS2_CHECK(kv_dtype == HS2_KV_FP8_E4M3, HS2_ERR_INVALID_ARG, "bad kv_dtype");
+  HS2_CHECK(Tq == 1 && q_start == kv_len - 1, HS2_ERR_UNSUPPORTED,
+            "FP8 decode takes Tq == 1 with q_start == kv_len - 1");
+  HS2_CHECK(k_scale && v_scale && aligned4(k_scale) && aligned4(v_scale), HS2_ERR_INVALID_ARG,
+            "FP8 KV needs 4-byte aligned k_scale and v_scale");
+  HS2_CHECK(kv_stride_tokens >= kv_len, HS2_ERR_INVALID_ARG, "kv_stride_tokens must be >= kv_len");
+  HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
+  return d == 256 ? decode_select<256>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
+                                       softmax_scale, O, idx, workspace, st, ctx)
+                  : decode_select<128>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
+                                       softmax_scale, O, idx, workspace, st, ctx);
+}
+
+hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, const int32_t* idx, int64_t Tq,
+                                   int64_t kv_len, int n_idx, int Hq, int d, float softmax_scale, void* O,
+                                   void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(Q && K && V && idx && O, HS2_ERR_INVALID_ARG, "null tensor pointer");
+  HS2_CHECK(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned4(idx), HS2_ERR_INVALID_ARG,
+            "Q, K, V, O must be 16-byte aligned and idx 4-byte aligned");
+  HS2_CHECK(Tq >= 1 && Tq < (1ll << 31) && kv_len >= 1 && n_idx >= 1, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(n_idx <= 2048, HS2_ERR_UNSUPPORTED, "n_idx must be <= 2048");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  Attn16Params p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = K;
+  p.V = V;
+  p.idx = idx;
+  p.n_idx = n_idx;
+  p.kv_len = kv_len;
+  p.kv_stride = 0;
+  p.H = Hq;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.splits = 1;
+  p.slots_per_split = n_idx;
+  p.final_out = 1;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? launch_attn16<256, false, false>(p, (int)Tq, st, ctx)
+                  : launch_attn16<128, false, false>(p, (int)Tq, st, ctx);
+}
+
+hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d, size_t* bytes) {
+  g_err[0] = 0;
+  HS2_CHECK(bytes, HS2_ERR_INVALID_ARG, "bytes is null");
+  HS2_CHECK(batch >= 1 && n_idx >= 1, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  DevCtx ctx;
+  int sms = 0;
+  hs2_status s = device_ctx(&ctx, &sms);
+  if (s != HS2_OK) return s;
+  const int splits = sparse_decode_splits(batch, n_idx, sms);
+  *bytes = splits > 1 ? up256((size_t)batch * splits * (32 + 16 * (size_t)d) * sizeof(float)) : 0;
+  return HS2_OK;
+}
+
+hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                                  const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                                  int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
+                                  float softmax_scale, void* O, void* workspace, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(Q && Kc && Vc && k_scale && v_scale && idx && O, HS2_ERR_INVALID_ARG, "null tensor pointer");
+  HS2_CHECK(aligned16(Q) && aligned16(Kc) && aligned16(Vc) && aligned16(O) && aligned4(idx) && aligned4(k_scale) &&
+                aligned4(v_scale),
+            HS2_ERR_INVALID_ARG, "misaligned pointer");
+  HS2_CHECK(kv_dtype == HS2_KV_FP8_E4M3, HS2_ERR_UNSUPPORTED, "sparse decode reads an FP8 E4M3 cache");
+  HS2_CHECK(batch >= 1 && kv_len >= 1 && n_idx >= 1 && kv_stride_tokens >= kv_len, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(n_idx <= 2048, HS2_ERR_UNSUPPORTED, "n_idx must be <= 2048");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
+  HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  size_t need = 0;
+  hs2_status s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need);
+  if (s != HS2_OK) return s;
+  HS2_CHECK(ws_bytes >= need && (need == 0 || (workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0))),
+            HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
+  DevCtx ctx;
+  int sms = 0;
+  if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
+  const int splits = sparse_decode_splits(batch, n_idx, sms);
+  Attn16Params p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = Kc;
+  p.V = Vc;
+  p.ks = k_scale;
+  p.vs = v_scale;
+  p.idx = idx;
+  p.n_idx = n_idx;
+  p.kv_len = kv_len;
+  p.kv_stride = kv_stride_tokens;
+  p.H = Hq;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.splits = splits;
+  p.slots_per_split = (n_idx + splits - 1) / splits;
+  p.final_out = splits == 1;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.part = static_cast<float*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = d == 256 ? launch_attn16<256, true, false>(p, batch * splits, st, ctx)
+               : launch_attn16<128, true, false>(p, batch * splits, st, ctx);
+  if (s != HS2_OK || splits == 1) return s;
+  return d == 256 ? launch_combine<256>(p.part, splits, Hq, p.O, nullptr, batch, st)
+                  : launch_combine<128>(p.part, splits, Hq, p.O, nullptr, batch, st);
+}
+
+hs2_status hs2_device_status(void* stream) {
+  g_err[0] = 0;
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned w = 0;
+  e = cudaMemcpyFromSymbol(&w, g_status_word, sizeof(w));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  if (w & ST_TIMEOUT) return fail(HS2_ERR_TIMEOUT, "a device-side wait gave up");
+  if (w & ST_DEVICE_CHECK) return fail(HS2_ERR_DEVICE_CHECK, "a device-side input check failed");
+  return HS2_OK;
+}
+
+hs2_status hs2_set_spin_limit(int64_t iterations) {
+  g_err[0] = 0;
+  HS2_CHECK(iterations >= 0, HS2_ERR_INVALID_ARG, "iterations must be >= 0");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HS2_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_spin[dev] = iterations;
+  return HS2_OK;
+}
+
+}  // extern "C"
