@@ -182,6 +182,19 @@ HS2_API hs2_status hs2_device_status(void* stream);
  */
 HS2_API hs2_status hs2_set_spin_limit(int64_t iterations);
 
+/*
+ * Kernel timing (instrumentation; no counterpart in the method).  While
+ * enabled on the calling host thread, every kernel the library launches is
+ * bracketed by CUDA events recorded on its launch stream.
+ *   hs2_profile_enable(1) starts a fresh record, hs2_profile_enable(0) stops.
+ *   hs2_profile_collect() synchronises on the recorded events and returns, in
+ *   launch order, up to max_n entries: names[i] (static strings owned by the
+ *   library) and ms[i] (device time of launch i).  *n gets the number recorded
+ *   (which may exceed max_n; at most 4096 are kept).  The record is cleared.
+ */
+HS2_API hs2_status hs2_profile_enable(int on);
+HS2_API hs2_status hs2_profile_collect(const char** names, float* ms, int max_n, int* n);
+
 #ifdef __cplusplus
 }
 #endif

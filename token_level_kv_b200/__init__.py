@@ -49,6 +49,8 @@ def _load() -> ctypes.CDLL:
         "hs2_sparse_attn_decode_workspace": ([I, I, I, I, ctypes.POINTER(Z)], I),
         "hs2_device_status": ([P], I),
         "hs2_set_spin_limit": ([L], I),
+        "hs2_profile_enable": ([I], I),
+        "hs2_profile_collect": ([ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(F), I, ctypes.POINTER(I)], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -60,7 +62,8 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv", "hs2_full_attn_select",
            "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
-           "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit")
+           "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit",
+           "hs2_profile_enable", "hs2_profile_collect")
 
 
 def _check(status: int) -> None:
@@ -178,6 +181,20 @@ def hs2_device_status(stream=None) -> int:
 
 def hs2_set_spin_limit(iterations: int) -> None:
     _check(lib.hs2_set_spin_limit(iterations))
+
+
+def hs2_profile_enable(on: bool) -> None:
+    """Bracket every library kernel launch of this host thread with CUDA events."""
+    _check(lib.hs2_profile_enable(1 if on else 0))
+
+
+def hs2_profile_collect(max_n: int = 4096):
+    """[(kernel name, device ms)] for the launches recorded since enable; clears the record."""
+    names = (ctypes.c_char_p * max_n)()
+    ms = (ctypes.c_float * max_n)()
+    n = ctypes.c_int(0)
+    _check(lib.hs2_profile_collect(names, ms, max_n, ctypes.byref(n)))
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, max_n))]
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor | None:

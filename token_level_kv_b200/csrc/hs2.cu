@@ -116,9 +116,39 @@ hs2_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint6
   return HS2_OK;
 }
 
-hs2_status after_launch(const char* what) {
+// ------------------------------------------------------------------ profiling
+constexpr int kMaxProf = 4096;
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+thread_local bool g_prof_on = false;
+thread_local int g_prof_n = 0;
+thread_local ProfRec g_prof[kMaxProf];
+thread_local int g_prof_events = 0;      // event pairs created so far (reused)
+
+// Records the "before" event of the next launch on stream st.
+void prof_begin(cudaStream_t st) {
+  if (!g_prof_on || g_prof_n >= kMaxProf) return;
+  ProfRec& r = g_prof[g_prof_n];
+  if (g_prof_n >= g_prof_events) {
+    cudaEventCreate(&r.a);
+    cudaEventCreate(&r.b);
+    ++g_prof_events;
+  }
+  cudaEventRecord(r.a, st);
+}
+
+hs2_status after_launch(const char* what, cudaStream_t st) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
+  if (g_prof_on) {
+    if (g_prof_n < kMaxProf) {
+      g_prof[g_prof_n].name = what;
+      cudaEventRecord(g_prof[g_prof_n].b, st);
+    }
+    ++g_prof_n;
+  }
   return HS2_OK;
 }
 
@@ -175,15 +205,17 @@ hs2_status launch_attn16(const Attn16Params& p, int grid, cudaStream_t st, const
   constexpr size_t smem = A16Layout<D, FP8>::SMEM;
   hs2_status s = set_smem(attn16_kernel<D, FP8, RANGE>, smem);
   if (s != HS2_OK) return s;
+  prof_begin(st);
   attn16_kernel<D, FP8, RANGE><<<grid, 128, smem, st>>>(p, ctx);
-  return after_launch("attn16_kernel");
+  return after_launch("attn16_kernel", st);
 }
 
 template <int D>
 hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
                           cudaStream_t st) {
+  prof_begin(st);
   attn16_combine_kernel<D><<<items, 256, 0, st>>>(part, splits, H, O, ml);
-  return after_launch("attn16_combine_kernel");
+  return after_launch("attn16_combine_kernel", st);
 }
 
 template <int D>
@@ -211,8 +243,9 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
   fp.ml = ml;
   fp.n_qtiles = (int)((Tq * Hq + 127) / 128);
   if ((s = set_smem(fa_fwd_kernel<D>, FaLayout<D>::SMEM)) != HS2_OK) return s;
+  prof_begin(st);
   fa_fwd_kernel<D><<<fp.n_qtiles, FA_THREADS, FaLayout<D>::SMEM, st>>>(mQ, mK, mV, fp, ctx);
-  if ((s = after_launch("fa_fwd_kernel")) != HS2_OK) return s;
+  if ((s = after_launch("fa_fwd_kernel", st)) != HS2_OK) return s;
 
   SgParams sp;
   sp.Tq = Tq;
@@ -227,12 +260,14 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
   sp.n_groups = (int)((Tq * Hq + 255) / 256);
   if (Hq == 16) {
     if ((s = set_smem(select_sigma_kernel<D, 16>, SgLayout<D>::SMEM)) != HS2_OK) return s;
+    prof_begin(st);
     select_sigma_kernel<D, 16><<<sp.n_groups, SG_THREADS, SgLayout<D>::SMEM, st>>>(mQ256, mK, sp, ctx);
   } else {
     if ((s = set_smem(select_sigma_kernel<D, 8>, SgLayout<D>::SMEM)) != HS2_OK) return s;
+    prof_begin(st);
     select_sigma_kernel<D, 8><<<sp.n_groups, SG_THREADS, SgLayout<D>::SMEM, st>>>(mQ256, mK, sp, ctx);
   }
-  if ((s = after_launch("select_sigma_kernel")) != HS2_OK) return s;
+  if ((s = after_launch("select_sigma_kernel", st)) != HS2_OK) return s;
 
   TopkParams tp;
   tp.sigma = sigma;
@@ -243,8 +278,9 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
   tp.topk = topk;
   tp.idx = idx;
   if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
+  prof_begin(st);
   topk_select_kernel<<<(unsigned)Tq, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
-  return after_launch("topk_select_kernel");
+  return after_launch("topk_select_kernel", st);
 }
 
 template <int D>
@@ -282,8 +318,9 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
   if (n_cand > 0) {
     dim3 g((unsigned)((n_cand + 255) / 256), (unsigned)batch);
+    prof_begin(st);
     decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld);
-    if ((s = after_launch("decode_sigma_kernel")) != HS2_OK) return s;
+    if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
   }
   TopkParams tp;
   tp.sigma = sigma;
@@ -294,8 +331,9 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   tp.topk = topk;
   tp.idx = idx;
   if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
+  prof_begin(st);
   topk_select_kernel<<<(unsigned)batch, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
-  return after_launch("topk_select_kernel");
+  return after_launch("topk_select_kernel", st);
 }
 
 }  // namespace
@@ -358,8 +396,9 @@ hs2_status hs2_bridge_kv(const void* hidden, int64_t rows, int hidden_dim, const
   p.num_tiles = (int)(2 * ((rows + BG_BM - 1) / BG_BM));
   if ((s = set_smem(bridge_gemm_kernel, BG_SMEM)) != HS2_OK) return s;
   const int grid = std::min(p.num_tiles, sms);
+  prof_begin(static_cast<cudaStream_t>(stream));
   bridge_gemm_kernel<<<grid, BG_THREADS, BG_SMEM, static_cast<cudaStream_t>(stream)>>>(mA, mWk, mWv, p, ctx);
-  return after_launch("bridge_gemm_kernel");
+  return after_launch("bridge_gemm_kernel", static_cast<cudaStream_t>(stream));
 }
 
 hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int64_t Tq, int64_t kv_len, int Hq,
@@ -536,6 +575,31 @@ hs2_status hs2_device_status(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "clear status word");
   if (w & ST_TIMEOUT) return fail(HS2_ERR_TIMEOUT, "a device-side wait gave up");
   if (w & ST_DEVICE_CHECK) return fail(HS2_ERR_DEVICE_CHECK, "a device-side input check failed");
+  return HS2_OK;
+}
+
+hs2_status hs2_profile_enable(int on) {
+  g_err[0] = 0;
+  g_prof_on = on != 0;
+  if (g_prof_on) g_prof_n = 0;
+  return HS2_OK;
+}
+
+hs2_status hs2_profile_collect(const char** names, float* ms, int max_n, int* n) {
+  g_err[0] = 0;
+  HS2_CHECK(n && (max_n <= 0 || (names && ms)), HS2_ERR_INVALID_ARG, "null output");
+  const int kept = std::min(g_prof_n, kMaxProf);
+  for (int i = 0; i < kept && i < max_n; ++i) {
+    cudaError_t e = cudaEventSynchronize(g_prof[i].b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, g_prof[i].a, g_prof[i].b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    names[i] = g_prof[i].name;
+    ms[i] = t;
+  }
+  *n = g_prof_n;
+  g_prof_n = 0;
   return HS2_OK;
 }
 
