@@ -121,6 +121,18 @@ def prefill_flops(T, H, d, window, topk, n_sparse):
     return full, sparse, n_sparse * sparse, sigma
 
 
+def reduce_max(value: float, device) -> float:
+    """Max over all ranks (the timing rule for N > 1); works for nccl and gloo."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(step_flops: float, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs one replica of the step."""
+    return world * step_flops / (max_ms * 1e-3) / 1e12
+
+
 def timed_steps(step, steps, flush, stream):
     """Per-step CUDA events on the launching stream, L2 flushed between steps."""
     ts = []
@@ -282,10 +294,8 @@ def run_ours(args, rank, world, dist):
         torch.distributed.barrier()
     ms = statistics.mean(step_ms)
     if dist:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = world * step_flops / (ms * 1e-3) / 1e12
+        ms = reduce_max(ms, dev)
+    value = weak_scaling_value(step_flops, world, ms)
     kern = per_kernel(prof)
     launches = len(prof)
 
@@ -342,10 +352,8 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         e_ms = statistics.mean(timed_steps(e2e_step, max(2, min(args.steps, 5)), lambda: None, stream))
         if dist:
-            tt = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        out["e2e"] = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+            e_ms = reduce_max(e_ms, dev)
+        out["e2e"] = {"value": weak_scaling_value(step_flops, world, e_ms), "unit": "TFLOP/s", "ms_per_step": e_ms,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del hin, din, hout
 
