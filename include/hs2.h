@@ -168,6 +168,36 @@ HS2_API hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq
                                             size_t* bytes);
 
 /*
+ * hs2_sparse_attn_decode without a workspace argument.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves -- e.g. a serving process whose device memory is
+ * all reserved up front by its own pool and handed to plugins as fixed
+ * buffers, or a decode loop that must not pay for cudaMalloc's implicit
+ * synchronisation.  Same arguments, results and errors as
+ * hs2_sparse_attn_decode, which it calls with its scratch instead of a
+ * caller's workspace.
+ *   - Scratch: one file-scope device array of HS2_STATIC_SCRATCH_BYTES
+ *     (8 MiB) that every GPU loading the library holds until the process
+ *     exits.  A call whose split partials need more than that (see
+ *     hs2_sparse_attn_decode_workspace) fails with HS2_ERR_UNSUPPORTED and
+ *     launches nothing.  Nothing is allocated, by this call or the library.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one array.  Its contents need no
+ *     clearing (each call writes every partial it reads), but calls whose
+ *     executions overlap on the GPU -- on different streams, or from
+ *     different host threads -- race on it and give wrong results.
+ */
+#define HS2_STATIC_SCRATCH_BYTES (8u << 20)
+HS2_API hs2_status hs2_sparse_attn_decode_static(const void* Q, const void* Kc, const void* Vc,
+                                         const float* k_scale, const float* v_scale,
+                                         hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                                         int64_t kv_stride_tokens, const int32_t* idx, int n_idx,
+                                         int Hq, int d, float softmax_scale, void* O,
+                                         void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the status word of the current
  * device: HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA if
  * the synchronisation itself failed).

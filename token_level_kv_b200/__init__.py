@@ -47,6 +47,7 @@ def _load() -> ctypes.CDLL:
         "hs2_sparse_attn_prefill": ([P, P, P, P, L, L, I, I, I, F, P, P], I),
         "hs2_sparse_attn_decode": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P, Z, P], I),
         "hs2_sparse_attn_decode_workspace": ([I, I, I, I, ctypes.POINTER(Z)], I),
+        "hs2_sparse_attn_decode_static": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P], I),
         "hs2_device_status": ([P], I),
         "hs2_set_spin_limit": ([L], I),
         "hs2_profile_enable": ([I], I),
@@ -63,7 +64,7 @@ lib = _load()
 EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv", "hs2_full_attn_select",
            "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
            "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit",
-           "hs2_profile_enable", "hs2_profile_collect")
+           "hs2_profile_enable", "hs2_profile_collect", "hs2_sparse_attn_decode_static")
 
 
 def _check(status: int) -> None:
@@ -172,6 +173,21 @@ def hs2_sparse_attn_decode(Q, Kc, Vc, k_scale, v_scale, idx, O, workspace=None, 
     _check(lib.hs2_sparse_attn_decode(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale), KV_FP8_E4M3, B,
                                       kv_len, stride, _ptr(idx), idx.shape[-1], H, d, scale, _ptr(O),
                                       _ptr(workspace), ws, _stream(stream)))
+
+
+def hs2_sparse_attn_decode_static(Q, Kc, Vc, k_scale, v_scale, idx, O, *, kv_len: int | None = None,
+                                  softmax_scale: float | None = None, stream=None) -> None:
+    """hs2_sparse_attn_decode for callers that cannot allocate device memory:
+    the split partials go to the library's own 8 MiB static device array
+    instead of a workspace.  Calls that overlap on the GPU share that array
+    and race; run them one after another."""
+    B, H, d = Q.shape
+    stride = Kc.shape[1]
+    kv_len = stride if kv_len is None else kv_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    _check(lib.hs2_sparse_attn_decode_static(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale),
+                                             KV_FP8_E4M3, B, kv_len, stride, _ptr(idx), idx.shape[-1], H, d,
+                                             scale, _ptr(O), _stream(stream)))
 
 
 def hs2_device_status(stream=None) -> int:

@@ -560,6 +560,54 @@ hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
                   : launch_combine<128>(p.part, splits, Hq, p.O, nullptr, batch, st);
 }
 
+}  // extern "C"
+
+// Scratch of hs2_sparse_attn_decode_static: the split partials of the sparse
+// decode live here instead of in a caller workspace.  Module scope, so every
+// device that loads the library holds these 8 MiB until the process exits.
+static __device__ __align__(256) float g_static_scratch[HS2_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+float* g_static_scratch_ptr[hs2::kMaxDevices];
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (the host-side symbol is only a stand-in, never a device pointer).
+hs2_status static_scratch_ptr(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return hs2::cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= hs2::kMaxDevices) return hs2::fail(HS2_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(hs2::g_mu);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return hs2::cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_static_scratch_ptr[dev];
+  return HS2_OK;
+}
+}  // namespace
+
+extern "C" {
+
+hs2_status hs2_sparse_attn_decode_static(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                                         const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                                         int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
+                                         float softmax_scale, void* O, void* stream) {
+  g_err[0] = 0;
+  size_t need = 0;
+  hs2_status s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need);
+  if (s != HS2_OK) return s;
+  HS2_CHECK(need <= HS2_STATIC_SCRATCH_BYTES, HS2_ERR_UNSUPPORTED,
+            "this batch needs %zu bytes of split scratch; the static array holds %u "
+            "(use hs2_sparse_attn_decode with a workspace)", need, (unsigned)HS2_STATIC_SCRATCH_BYTES);
+  float* scratch = nullptr;
+  if ((s = static_scratch_ptr(&scratch)) != HS2_OK) return s;
+  return hs2_sparse_attn_decode(Q, Kc, Vc, k_scale, v_scale, kv_dtype, batch, kv_len, kv_stride_tokens, idx,
+                                n_idx, Hq, d, softmax_scale, O, scratch, HS2_STATIC_SCRATCH_BYTES, stream);
+}
+
 hs2_status hs2_device_status(void* stream) {
   g_err[0] = 0;
   DevCtx ctx;
