@@ -251,6 +251,16 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
+    if args.only_decode:
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+        def flush_only():
+            flush_buf.zero_()
+            flush_rd.max()
+        if rank == 0:
+            print(json.dumps({"decode": bench_decode(hs2, dev, stream, flush_only, peaks, peak_src, args)}), flush=True)
+        return
     w = WORKLOAD
     T, H, d, W, k = w["T"], w["H"], w["d"], w["window"], w["topk"]
     case = synth.make_prefill_case(T, H, d, W, k, w["n_sparse"], n_needles=w["n_needles"], scale=w["scale"],
@@ -260,9 +270,13 @@ def run_ours(args, rank, world, dist):
     Os = [torch.empty_like(O) for _ in range(w["n_sparse"])]
     ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_BF16, 1, T, T, H, d, W, k), dev)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
     def flush():
+        # write 256 MiB (> 126 MB L2), then read another 256 MiB so the timed
+        # call does not pay for writing the flush's dirty lines back
         flush_buf.zero_()
+        flush_rd.max()
 
     def step():
         hs2.hs2_full_attn_select(case.Q, case.K, case.V, O, idx, ws, window=W, topk=k)
@@ -410,12 +424,16 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
     n = max(3, args.steps)
     hs2.hs2_profile_enable(True)
     t_full = timed_steps(full, n, flush, stream)
+    prof_full = per_kernel(hs2.hs2_profile_collect())
     t_sp = [timed_steps(lambda l=l: sparse(l), n, flush, stream) for l in range(c["n_sparse"])]
-    t_warm = timed_steps(lambda: [sparse(l) for l in range(c["n_sparse"])], n, lambda: None, stream)
-    prof = per_kernel(hs2.hs2_profile_collect())
+    prof_sp = per_kernel(hs2.hs2_profile_collect())
     hs2.hs2_profile_enable(False)
+    t_warm = timed_steps(lambda: [sparse(l) for l in range(c["n_sparse"])], n, lambda: None, stream)
+    prof = {"full_select_call": prof_full, "sparse_call": prof_sp}
     ms_full = statistics.median(t_full)
     ms_sp = [statistics.median(t) for t in t_sp]
+    # device time of the sparse-decode kernels alone (library events around each launch)
+    sp_kernel_ms = sum(v["total_ms"] for v in prof_sp.values()) / (n * c["n_sparse"])
     full_bytes = B * N * (2 * d + 8) + B * H * d * 2 * 2 + B * (W + k) * 4
     sp_bytes = B * ((W + k) * (2 * d + 8 + 4) + 2 * H * d * 2)
     step_ms = ms_full + sum(ms_sp)
@@ -427,6 +445,9 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
         "tok_s": B / (step_ms * 1e-3), "step_ms": step_ms,
         "full_select_ms": ms_full, "full_select_gbs": full_gbs, "full_select_frac": full_gbs / peaks["hbm_gbs"],
         "sparse_ms": ms_sp, "sparse_gbs": sp_gbs, "sparse_frac": sp_gbs / peaks["hbm_gbs"],
+        "sparse_kernel_ms": sp_kernel_ms,
+        "sparse_kernel_gbs": sp_bytes / (sp_kernel_ms * 1e-3) / 1e9,
+        "sparse_kernel_frac": sp_bytes / (sp_kernel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "sparse_tok_s_per_layer": B / (statistics.mean(ms_sp) * 1e-3),
         "sparse_warm_chain_ms": statistics.median(t_warm),
         "algorithmic_bytes": {"full_select": full_bytes, "sparse_per_layer": sp_bytes},
@@ -476,8 +497,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=48)
     ap.add_argument("--T", type=int, default=None, help="override the prefill length (small profiling cases)")
+    ap.add_argument("--decode-N", type=int, default=None, help="override the decode context (small profiling cases)")
+    ap.add_argument("--only-decode", action="store_true", help="run the decode measurement only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    if args.decode_N:
+        DECODE["N"] = args.decode_N
     if args.T:
         WORKLOAD["T"] = args.T
         WORKLOAD["n_needles"] = min(WORKLOAD["n_needles"], max(0, args.T // 512))

@@ -209,3 +209,27 @@ def test_bounded_wait_gives_up_and_context_survives(hs2):
     bad, _ = bf16_rule(K[:300].cpu(), oracle.bridge_rows(c.hidden[:300], c.Wk[0]),
                        abs_dot(c.hidden[:300], c.Wk[0]))
     assert bad == 0
+
+
+def test_fp8_widening_is_exact_for_every_code(hs2):
+    """One selected key: its probability is 1 and O = v_scale * E4M3(V row), so
+    the bf16 output reproduces all 254 finite codes (subnormals included)."""
+    d = 256
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    codes[0x7F] = 0
+    codes[0xFF] = 0                            # the two NaN codes are not stored
+    Vc = torch.zeros(1, 16, d, dtype=torch.uint8)
+    Vc[0, 3] = codes
+    Kc = torch.randint(0, 0x7E, (1, 16, d), dtype=torch.uint8)
+    ks = torch.ones(1, 16)
+    vs = torch.ones(1, 16)
+    Q = synth.normal_bf16(0, 1, (1, 16, d))
+    idx = torch.full((1, 16), -1, dtype=torch.int32)
+    idx[0, 0] = 3
+    O = torch.empty(1, 16, d, dtype=torch.bfloat16, device="cuda")
+    ws = hs2.workspace(hs2.hs2_sparse_attn_decode_workspace(1, 16, 16, d))
+    hs2.hs2_sparse_attn_decode(Q.cuda(), Kc.cuda(), Vc.cuda(), ks.cuda(), vs.cuda(), idx.cuda(), O, ws)
+    assert hs2.hs2_device_status() == 0
+    want = torch.from_numpy(oracle.e4m3_decode(codes.numpy()))
+    for h in range(16):
+        assert torch.equal(O[0, h].double().cpu(), want)

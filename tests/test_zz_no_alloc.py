@@ -29,7 +29,7 @@ def _case(seed, B, N):
 
 def test_static_scratch_matches_workspace_path_two_calls_in_a_row():
     import token_level_kv_b200 as hs2
-    B, N = 70, 3000                      # several splits per sequence: the scratch is used
+    B, N = 4, 3000                       # small batch: more splits than a cluster, so the scratch is used
     assert hs2.hs2_sparse_attn_decode_workspace(B, 1152, 16, 256) > 0
     cases = [_case(21, B, N), _case(22, B, N)]
     got = []

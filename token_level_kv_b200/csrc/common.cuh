@@ -257,6 +257,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
   return pack_bf16x2(f.x, f.y);
 }
 
+// Two E4M3 codes (low byte first) -> two f16, exactly (one instruction).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 // fp32 pair -> two E4M3 codes, round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t r;

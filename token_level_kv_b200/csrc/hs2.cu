@@ -16,6 +16,7 @@
 #include "attn16.cuh"
 #include "bridge_gemm.cuh"
 #include "common.cuh"
+#include "decode_attn.cuh"
 #include "fa_fwd.cuh"
 #include "select_sigma.cuh"
 #include "topk.cuh"
@@ -193,29 +194,65 @@ DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d) {
   return w;
 }
 
+// CTAs per sequence of the sparse decode.  Up to 8 they form one thread-block
+// cluster and merge in distributed shared memory (no workspace); a batch too
+// small to fill the GPU that way uses more splits and a workspace.
+constexpr int kMaxCluster = 8;
 int sparse_decode_splits(int batch, int n_idx, int num_sms) {
-  int s = (num_sms + batch - 1) / batch;
   const int max_s = std::max(1, (n_idx + 63) / 64);
-  return std::max(1, std::min(s, max_s));
+  int s = num_sms / batch;
+  if (s <= kMaxCluster) return std::max(1, std::min(s, std::min(max_s, kMaxCluster)));
+  return std::min((num_sms + batch - 1) / batch, max_s);
 }
 
 // ------------------------------------------------------------------ launches
-template <int D, bool FP8, bool RANGE>
-hs2_status launch_attn16(const Attn16Params& p, int grid, cudaStream_t st, const DevCtx& ctx) {
-  constexpr size_t smem = A16Layout<D, FP8>::SMEM;
-  hs2_status s = set_smem(attn16_kernel<D, FP8, RANGE>, smem);
-  if (s != HS2_OK) return s;
-  prof_begin(st);
-  attn16_kernel<D, FP8, RANGE><<<grid, 128, smem, st>>>(p, ctx);
-  return after_launch("attn16_kernel", st);
-}
-
 template <int D>
 hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
                           cudaStream_t st) {
   prof_begin(st);
   attn16_combine_kernel<D><<<items, 256, 0, st>>>(part, splits, H, O, ml);
   return after_launch("attn16_combine_kernel", st);
+}
+
+template <int D>
+hs2_status launch_sparse_prefill(const Attn16Params& p, int grid, cudaStream_t st, const DevCtx& ctx) {
+  hs2_status s = set_smem(sparse_prefill_kernel<D>, SpfLayout<D>::SMEM);
+  if (s != HS2_OK) return s;
+  prof_begin(st);
+  sparse_prefill_kernel<D><<<grid, 128, SpfLayout<D>::SMEM, st>>>(p, ctx);
+  return after_launch("sparse_prefill_kernel", st);
+}
+
+template <int D>
+hs2_status launch_decode_parts(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
+  hs2_status s = set_smem(decode_attn_kernel<D, false, true>, DecLayout<D>::SMEM);
+  if (s != HS2_OK) return s;
+  prof_begin(st);
+  decode_attn_kernel<D, false, true><<<batch * p.splits, DecLayout<D>::NW * 32, DecLayout<D>::SMEM, st>>>(p, ctx);
+  return after_launch("decode_attn_kernel", st);
+}
+
+// One thread-block cluster of p.splits CTAs per sequence.
+template <int D>
+hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
+  hs2_status s = set_smem(decode_attn_kernel<D, false, false>, DecLayout<D>::SMEM);
+  if (s != HS2_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(batch * p.splits));
+  cfg.blockDim = dim3(DecLayout<D>::NW * 32);
+  cfg.dynamicSmemBytes = DecLayout<D>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  prof_begin(st);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<D, false, false>, p, ctx);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_attn_kernel)");
+  return after_launch("decode_attn_kernel", st);
 }
 
 template <int D>
@@ -293,27 +330,26 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   float* part = reinterpret_cast<float*>(b + w.logits);
   float* ml = reinterpret_cast<float*>(b + w.logits + w.part);
   float* sigma = reinterpret_cast<float*>(b + w.logits + w.part + w.ml);
-  Attn16Params p{};
+  DecParams p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
-  p.K = K;
-  p.V = V;
+  p.K = static_cast<const uint8_t*>(K);
+  p.V = static_cast<const uint8_t*>(V);
   p.ks = ks;
   p.vs = vs;
-  p.idx = nullptr;
-  p.n_idx = 0;
   p.kv_len = kv_len;
   p.kv_stride = kv_stride;
   p.H = Hq;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.splits = w.splits;
-  p.slots_per_split = kDecodeKeysPerSplit;
-  p.final_out = 0;
-  p.O = nullptr;
+  p.per_split = kDecodeKeysPerSplit;
   p.part = part;
   p.logits = logits;
   p.logit_ld = w.ld;
-  hs2_status s = launch_attn16<D, true, true>(p, batch * w.splits, st, ctx);
+  hs2_status s = set_smem(decode_attn_kernel<D, true, true>, DecLayout<D>::SMEM);
   if (s != HS2_OK) return s;
+  prof_begin(st);
+  decode_attn_kernel<D, true, true><<<batch * w.splits, DecLayout<D>::NW * 32, DecLayout<D>::SMEM, st>>>(p, ctx);
+  if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
   if ((s = launch_combine<D>(part, w.splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
   if (n_cand > 0) {
@@ -476,8 +512,7 @@ hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, 
   HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
   HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
   DevCtx ctx;
-  hs2_status s = device_ctx(&ctx, nullptr);
-  if (s != HS2_OK) return s;
+  hs2_status s;
   Attn16Params p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.K = K;
@@ -485,16 +520,15 @@ hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, 
   p.idx = idx;
   p.n_idx = n_idx;
   p.kv_len = kv_len;
-  p.kv_stride = 0;
   p.H = Hq;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.splits = 1;
-  p.slots_per_split = n_idx;
-  p.final_out = 1;
   p.O = static_cast<__nv_bfloat16*>(O);
+  p.n_rows = Tq;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 256 ? launch_attn16<256, false, false>(p, (int)Tq, st, ctx)
-                  : launch_attn16<128, false, false>(p, (int)Tq, st, ctx);
+  int sms = 0;
+  if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
+  const int grid = (int)std::min<int64_t>((Tq + 3) / 4, sms);
+  return d == 256 ? launch_sparse_prefill<256>(p, grid, st, ctx) : launch_sparse_prefill<128>(p, grid, st, ctx);
 }
 
 hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d, size_t* bytes) {
@@ -507,7 +541,7 @@ hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d,
   hs2_status s = device_ctx(&ctx, &sms);
   if (s != HS2_OK) return s;
   const int splits = sparse_decode_splits(batch, n_idx, sms);
-  *bytes = splits > 1 ? up256((size_t)batch * splits * (32 + 16 * (size_t)d) * sizeof(float)) : 0;
+  *bytes = splits > kMaxCluster ? up256((size_t)batch * splits * (32 + 16 * (size_t)d) * sizeof(float)) : 0;
   return HS2_OK;
 }
 
@@ -535,10 +569,10 @@ hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
   int sms = 0;
   if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
   const int splits = sparse_decode_splits(batch, n_idx, sms);
-  Attn16Params p{};
+  DecParams p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
-  p.K = Kc;
-  p.V = Vc;
+  p.K = static_cast<const uint8_t*>(Kc);
+  p.V = static_cast<const uint8_t*>(Vc);
   p.ks = k_scale;
   p.vs = v_scale;
   p.idx = idx;
@@ -548,16 +582,17 @@ hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
   p.H = Hq;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.splits = splits;
-  p.slots_per_split = (n_idx + splits - 1) / splits;
-  p.final_out = splits == 1;
+  p.per_split = (n_idx + splits - 1) / splits;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.part = static_cast<float*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = d == 256 ? launch_attn16<256, true, false>(p, batch * splits, st, ctx)
-               : launch_attn16<128, true, false>(p, batch * splits, st, ctx);
-  if (s != HS2_OK || splits == 1) return s;
-  return d == 256 ? launch_combine<256>(p.part, splits, Hq, p.O, nullptr, batch, st)
-                  : launch_combine<128>(p.part, splits, Hq, p.O, nullptr, batch, st);
+  if (splits > kMaxCluster) {
+    s = d == 256 ? launch_decode_parts<256>(p, batch, st, ctx) : launch_decode_parts<128>(p, batch, st, ctx);
+    if (s != HS2_OK) return s;
+    return d == 256 ? launch_combine<256>(p.part, splits, Hq, p.O, nullptr, batch, st)
+                    : launch_combine<128>(p.part, splits, Hq, p.O, nullptr, batch, st);
+  }
+  return d == 256 ? launch_decode_cluster<256>(p, batch, st, ctx) : launch_decode_cluster<128>(p, batch, st, ctx);
 }
 
 }  // extern "C"
