@@ -283,43 +283,32 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
   }
 }
 
-// Merge split partials: m = max m_s, l = sum l_s 2^(m_s-m), O = sum O_s 2^(m_s-m) / l.
+// Merge split partials of one (item, head) per CTA, one output dim per
+// thread: m = max m_s, l = sum l_s 2^(m_s-m), O = sum O_s 2^(m_s-m) / l.
 // Also stores (m, l) per head (log2 units) for the selection pass.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(D)
 attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, float* ml) {
-  const int item = blockIdx.x;
+  const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
   const float* base = part + (int64_t)item * splits * (32 + 16 * D);
-  __shared__ float sM[16], sL[16];
-  if (threadIdx.x < 16) {
-    const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, base[s * (32 + 16 * D) + h]);
-    float Lsum = 0.f;
-    if (M != -INFINITY)
-      for (int s = 0; s < splits; ++s) {
-        const float ms = base[s * (32 + 16 * D) + h];
-        if (ms != -INFINITY) Lsum += base[s * (32 + 16 * D) + 16 + h] * fast_exp2(ms - M);
-      }
-    sM[h] = M;
-    sL[h] = Lsum;
-    if (ml != nullptr && h < H) {
-      ml[((int64_t)item * H + h) * 2] = M;
-      ml[((int64_t)item * H + h) * 2 + 1] = Lsum;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, base[s * (32 + 16 * D) + h]);
+  float Ls = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float* ps = base + s * (32 + 16 * D);
+      const float ms = ps[h];
+      if (ms == -INFINITY) continue;
+      const float f = fast_exp2(ms - M);
+      Ls += ps[16 + h] * f;
+      acc += ps[32 + h * D + c] * f;
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < H * D; e += blockDim.x) {
-    const int h = e / D, c = e % D;
-    const float M = sM[h];
-    float acc = 0.f;
-    if (M != -INFINITY)
-      for (int s = 0; s < splits; ++s) {
-        const float ms = base[s * (32 + 16 * D) + h];
-        if (ms != -INFINITY) acc += base[s * (32 + 16 * D) + 32 + h * D + c] * fast_exp2(ms - M);
-      }
-    O[((int64_t)item * H + h) * D + c] = __float2bfloat16_rn(sL[h] > 0.f ? acc / sL[h] : 0.f);
+  if (c == 0 && ml != nullptr) {
+    ml[((int64_t)item * H + h) * 2] = M;
+    ml[((int64_t)item * H + h) * 2 + 1] = Ls;
   }
+  O[((int64_t)item * H + h) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
 }
 
 // Decode selection score: sigma[b, j] = sum_h 2^(x_hj - m_h) / l_h for the

@@ -8,9 +8,13 @@
 // Key j of sequence b is E4M3(K[b,j,:]) * k_scale[b,j], likewise V.
 //
 // Design (sm_100a), HBM-bound: everything serves bytes in flight.
-//   * 4 warps per CTA; each warp streams 16-key chunks through its own
-//     4-stage cp.async ring (3 chunks in flight), raw FP8 rows at a padded
-//     stride so the fragment loads below are bank-conflict free.
+//   * One producer warp streams 16-key chunks into a shared ring of NS stages
+//     (cp.async, completion tracked by cp.async.mbarrier.arrive on the stage's
+//     mbarrier), so almost the whole ring is in flight whatever the consumers
+//     are doing; NC consumer warps take chunk i from stage i % NS (consumer
+//     i % NC) and hand the stage back through its empty barrier.  Raw FP8
+//     rows sit at a padded stride so the fragment loads below are
+//     bank-conflict free.
 //   * The products run on mma.sync m16n8k16 in f16 with fp32 accumulation
 //     (the heads are M): every E4M3 code is an f16, so one cvt.rn.f16x2.e4m3x2
 //     widens two codes exactly.  Q enters in f16 after an exact power-of-two
@@ -32,7 +36,9 @@
 //     into key pairs of one dimension, and one cvt per pair widens them.  The
 //     O columns of a fragment are thus dims c0 + 2n + parity, a fixed
 //     permutation of d undone when the partial is written.
-//   * 6 warps per CTA, each with a 3-stage ring.
+//   * The index slice is copied to shared memory alongside the Q loads, so the
+//     first K/V requests leave after one round trip; Q is converted while
+//     they are in flight.
 //   * Online softmax in base 2 with a lazy rescale: the reference max moves
 //     only when a row's max grows by more than 2^8.
 //   * a7 (RANGE): the CTA owns one split of a sequence's keys, writes every
@@ -55,25 +61,26 @@ namespace cg = cooperative_groups;
 
 template <int D>
 struct DecLayout {
-  static constexpr int NW = 6;                      // warps per CTA
+  static constexpr int NC = 7;                      // consumer warps (8 warps with the producer)
+  static constexpr int NT = (NC + 1) * 32;          // + one producer warp
+  static constexpr int NS = 20;                     // ring stages (16 keys each)
   static constexpr int CH = 16;
-  static constexpr int NST = 3;
   static constexpr int KROW = D + 16;               // padded raw K row
   static constexpr int VROW = D + 16;               // padded raw V row (conflict-free ldmatrix)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + CH * KROW;
   static constexpr int OFF_KS = OFF_V + CH * VROW;
   static constexpr int OFF_VS = OFF_KS + CH * 4;
-  static constexpr int OFF_POS = OFF_VS + CH * 4;
-  static constexpr int STAGE = OFF_POS + CH * 4;
-  static constexpr int WARP = NST * STAGE;
-  static constexpr int QROW = 2 * D + 16;           // padded bf16 Q row
+  static constexpr int STAGE = OFF_VS + CH * 4;
+  static constexpr int QROW = 2 * D + 16;           // padded f16 Q row
   static constexpr int Q_BYTES = 16 * QROW;
   static constexpr int PART = (32 + 16 * D) * 4;    // one (m, l, O) partial
-  static constexpr int IDX = 2048 * 4;             // the CTA's index slice
-  static constexpr int OFF_IDX = Q_BYTES + NW * WARP;
-  static constexpr int MAIN = OFF_IDX + IDX;
-  static constexpr int MERGE = Q_BYTES + NW * PART + PART;
+  static constexpr int OFF_RING = Q_BYTES;
+  static constexpr int IDX = 2048 * 4;              // the CTA's index slice
+  static constexpr int OFF_IDX = OFF_RING + NS * STAGE;
+  static constexpr int OFF_BAR = OFF_IDX + IDX;
+  static constexpr int MAIN = OFF_BAR + 2 * NS * 8;
+  static constexpr int MERGE = Q_BYTES + NC * PART + PART;
   static constexpr size_t SMEM = (MAIN > MERGE ? MAIN : MERGE) + 128;
 };
 
@@ -98,7 +105,7 @@ struct DecParams {
 };
 
 template <int D, bool RANGE, bool PARTIALS>
-__global__ void __launch_bounds__(DecLayout<D>::NW * 32, 1)
+__global__ void __launch_bounds__(DecLayout<D>::NT, 1)
 decode_attn_kernel(DecParams p, DevCtx ctx) {
   using L = DecLayout<D>;
   extern __shared__ __align__(128) uint8_t smem_dec[];
@@ -107,29 +114,121 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
   const int g = lane >> 2, t = lane & 3;
   const int b = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;
+  uint8_t* ring = smem + L::OFF_RING;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + L::NS;
 
-  // ---- Q rows (zero beyond H) -> f16 with an exact power-of-two prescale
-  uint8_t* sQ = smem;
-  __shared__ float red_max[L::NW];
-  float qscale_inv;
+  const int64_t s_begin = (int64_t)split * p.per_split;
+  const int64_t total = RANGE ? p.kv_len : (int64_t)p.n_idx;
+  const int64_t s_end = min(total, s_begin + p.per_split);
+  const int n_chunks = s_end > s_begin ? (int)((s_end - s_begin + L::CH - 1) / L::CH) : 0;
+  const int64_t seq = (int64_t)b * p.kv_stride;
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + L::OFF_IDX);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::NS; ++s) {
+      mbar_init(&full[s], 32);             // the producer lanes' cp.async arrivals
+      mbar_init(&empty[s], 1);             // the consuming warp
+    }
+    fence_barrier_init();
+  }
+  // ---- start-up: the index slice -> shared memory (cp.async, then each
+  // thread checks the entries it copied) while Q comes into registers
+  if (!RANGE) {
+    for (int64_t i = threadIdx.x; i < s_end - s_begin; i += blockDim.x)
+      cp_async4(smem_u32(sidx + i), p.idx + (int64_t)b * p.n_idx + s_begin + i, true);
+  }
+  cp_async_commit();
+  constexpr int QV = 16 * D / 8;                     // uint4 groups of the 16 Q rows
+  constexpr int QPT = (QV + L::NT - 1) / L::NT;
+  uint4 qraw[QPT];
+  float mx = 0.f;
   {
     const __nv_bfloat16* q = p.Q + (int64_t)b * p.H * D;
-    float mx = 0.f;
-    for (int e = threadIdx.x; e < p.H * D; e += blockDim.x) mx = fmaxf(mx, fabsf(__bfloat162float(q[e])));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red_max[warp] = mx;
-    __syncthreads();
-    for (int w = 0; w < L::NW; ++w) mx = fmaxf(mx, red_max[w]);
-    const int ex = mx > 0.f ? 14 - ilogbf(mx) : 0;        // mx * 2^ex in [2^14, 2^15)
+    for (int k = 0; k < QPT; ++k) {
+      const int u = threadIdx.x + k * L::NT;
+      const int r = u / (D / 8), un = u % (D / 8);
+      qraw[k] = make_uint4(0, 0, 0, 0);
+      if (u < QV && r < p.H) qraw[k] = *reinterpret_cast<const uint4*>(q + r * D + un * 8);
+      const uint32_t* rw = reinterpret_cast<const uint32_t*>(&qraw[k]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[i]));
+        mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  __shared__ float red_max[L::NC + 1];
+  if (lane == 0) red_max[warp] = mx;
+  cp_async_wait<0>();
+  if (!RANGE) {
+    for (int64_t i = threadIdx.x; i < s_end - s_begin; i += blockDim.x) {
+      const int32_t v = sidx[i];
+      if (v < -1 || v >= p.kv_len) {
+        report(ctx, ST_DEVICE_CHECK);
+        sidx[i] = -1;
+      }
+    }
+  }
+  __syncthreads();                                   // barriers, index slice, maxima
+
+  uint8_t* sQ = smem;
+  // ------------------------------------------------------------ producer
+  // chunk i -> stage i % NS; the first ring round needs no empty wait, so it
+  // is issued before the block-wide barrier below (nothing can block there)
+  constexpr int UPR = D / 16;                        // 16-byte units per FP8 row
+  const int pkey = lane >> 1, pu0 = (lane & 1) * (UPR / 2);
+  auto produce = [&](int i) -> bool {
+    const int s = i % L::NS;
+    if (!mbar_wait(&empty[s], (uint32_t)(((i / L::NS) & 1) ^ 1), ctx)) return false;
+    uint8_t* st = ring + s * L::STAGE;
+    const int64_t sl = s_begin + (int64_t)i * L::CH + pkey;
+    const int32_t pk = sl < s_end ? (RANGE ? (int32_t)sl : sidx[sl - s_begin]) : -1;
+    const int64_t row = seq + (pk < 0 ? 0 : pk);
+    const uint8_t* ksrc = p.K + row * D + pu0 * 16;
+    const uint8_t* vsrc = p.V + row * D + pu0 * 16;
+    const uint32_t kdst = smem_u32(st + L::OFF_K + pkey * L::KROW + pu0 * 16);
+    const uint32_t vdst = smem_u32(st + L::OFF_V + pkey * L::VROW + pu0 * 16);
+#pragma unroll
+    for (int u = 0; u < UPR / 2; ++u) {
+      cp_async16(kdst + u * 16, ksrc + u * 16, pk >= 0);
+      cp_async16(vdst + u * 16, vsrc + u * 16, pk >= 0);
+    }
+    if ((lane & 1) == 0) {
+      cp_async4(smem_u32(st + L::OFF_KS + pkey * 4), p.ks + row, pk >= 0);
+      cp_async4(smem_u32(st + L::OFF_VS + pkey * 4), p.vs + row, pk >= 0);
+    }
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+    return true;
+  };
+  const int first_round = min(n_chunks, L::NS);
+  bool prod_ok = true;
+  if (warp == L::NC)
+    for (int i = 0; i < first_round && prod_ok; ++i) prod_ok = produce(i);
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float qscale_inv = 1.f;
+  // ---- Q -> f16 with an exact power-of-two prescale (largest element in
+  // [2^14, 2^15)), written while the first chunks are in flight
+  {
+    float m = 0.f;
+    for (int w = 0; w <= L::NC; ++w) m = fmaxf(m, red_max[w]);
+    const int ex = m > 0.f ? 14 - ilogbf(m) : 0;
     const float qs = ldexpf(1.f, ex);
     qscale_inv = ldexpf(1.f, -ex);
-    for (int u = threadIdx.x; u < 16 * D / 8; u += blockDim.x) {
-      const int r = u / (D / 8), un = u % (D / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < p.H) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(q + r * D + un * 8);
-        const uint32_t* rw = reinterpret_cast<const uint32_t*>(&raw);
+#pragma unroll
+    for (int k = 0; k < QPT; ++k) {
+      const int u = threadIdx.x + k * L::NT;
+      if (u < QV) {
+        const int r = u / (D / 8), un = u % (D / 8);
+        const uint32_t* rw = reinterpret_cast<const uint32_t*>(&qraw[k]);
+        uint4 v;
         uint32_t* ow = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -137,86 +236,30 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
           __half2 h = __floats2half2_rn(f.x * qs, f.y * qs);
           ow[i] = *reinterpret_cast<uint32_t*>(&h);
         }
-      }
-      *reinterpret_cast<uint4*>(sQ + r * L::QROW + un * 16) = v;
-    }
-  }
-
-  const int64_t s_begin = (int64_t)split * p.per_split;
-  const int64_t total = RANGE ? p.kv_len : (int64_t)p.n_idx;
-  const int64_t s_end = min(total, s_begin + p.per_split);
-  const int n_chunks = s_end > s_begin ? (int)((s_end - s_begin + L::CH - 1) / L::CH) : 0;
-  const int my_n = warp < n_chunks ? (n_chunks - warp + L::NW - 1) / L::NW : 0;
-  const int64_t seq = (int64_t)b * p.kv_stride;
-  int32_t* sidx = reinterpret_cast<int32_t*>(smem + L::OFF_IDX);
-  if (!RANGE) {
-    for (int64_t i = threadIdx.x; i < s_end - s_begin; i += blockDim.x) {
-      int32_t v = p.idx[(int64_t)b * p.n_idx + s_begin + i];
-      if (v < -1 || v >= p.kv_len) {
-        report(ctx, ST_DEVICE_CHECK);
-        v = -1;
-      }
-      sidx[i] = v;
-    }
-  }
-  uint8_t* wb = smem + L::Q_BYTES + warp * L::WARP;
-
-  auto issue = [&](int s, int chunk) {
-    uint8_t* st = wb + s * L::STAGE;
-    const int64_t sl = s_begin + (int64_t)chunk * L::CH + lane;
-    int32_t pos = -1;
-    if (lane < L::CH && sl < s_end) {
-      pos = RANGE ? (int32_t)sl : sidx[sl - s_begin];
-    }
-    if (lane < L::CH) reinterpret_cast<int32_t*>(st + L::OFF_POS)[lane] = pos;
-    {
-      // lane -> key lane/2, half lane%2 of its row: UPR/2 16-byte copies each for K and V
-      constexpr int UPR = D / 16;
-      const int key = lane >> 1, u0 = (lane & 1) * (UPR / 2);
-      const int32_t pk = __shfl_sync(0xffffffffu, pos, key);
-      const int64_t row = seq + (pk < 0 ? 0 : pk);
-      const uint8_t* ksrc = p.K + row * D + u0 * 16;
-      const uint8_t* vsrc = p.V + row * D + u0 * 16;
-      const uint32_t kdst = smem_u32(st + L::OFF_K + key * L::KROW + u0 * 16);
-      const uint32_t vdst = smem_u32(st + L::OFF_V + key * L::VROW + u0 * 16);
-#pragma unroll
-      for (int u = 0; u < UPR / 2; ++u) {
-        cp_async16(kdst + u * 16, ksrc + u * 16, pk >= 0);
-        cp_async16(vdst + u * 16, vsrc + u * 16, pk >= 0);
+        *reinterpret_cast<uint4*>(sQ + r * L::QROW + un * 16) = v;
       }
     }
-    if (lane < L::CH) {
-      const int64_t row = seq + (pos < 0 ? 0 : pos);
-      cp_async4(smem_u32(st + L::OFF_KS + lane * 4), p.ks + row, pos >= 0);
-      cp_async4(smem_u32(st + L::OFF_VS + lane * 4), p.vs + row, pos >= 0);
-    }
-  };
-
-  float o[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  __syncthreads();                       // Q and the index slice are in shared memory
-
-#pragma unroll
-  for (int s = 0; s < L::NST - 1; ++s) {
-    if (s < my_n) issue(s, warp + L::NW * s);
-    cp_async_commit();
   }
-  const uint32_t qa = smem_u32(sQ);
-  for (int it = 0; it < my_n; ++it) {
-    {
-      const int nxt = it + L::NST - 1;
-      if (nxt < my_n) issue(nxt % L::NST, warp + L::NW * nxt);
-      cp_async_commit();
-    }
-    cp_async_wait<L::NST - 1>();
-    __syncwarp();
-    const uint8_t* st = wb + (it % L::NST) * L::STAGE;
-    const int32_t* spos = reinterpret_cast<const int32_t*>(st + L::OFF_POS);
-    const float* sks = reinterpret_cast<const float*>(st + L::OFF_KS);
-    const float* svs = reinterpret_cast<const float*>(st + L::OFF_VS);
+  __syncthreads();                                   // Q in shared memory
 
+  if (warp == L::NC) {
+    for (int i = first_round; i < n_chunks && prod_ok; ++i) prod_ok = produce(i);
+    asm volatile("cp.async.wait_all;" ::: "memory");  // every issued copy lands before the merge reuses the ring
+  } else {
+    // ------------------------------------------------------------ consumers
+    for (int i = warp; i < n_chunks; i += L::NC) {
+      const int slot = i % L::NS;
+      if (!mbar_wait(&full[slot], (uint32_t)((i / L::NS) & 1), ctx)) break;
+      const uint8_t* st = ring + slot * L::STAGE;
+      const float* sks = reinterpret_cast<const float*>(st + L::OFF_KS);
+      const float* svs = reinterpret_cast<const float*>(st + L::OFF_VS);
+      // positions of this thread's keys 2t, 2t+1, 8+2t, 9+2t (-1: empty slot)
+      int32_t kpos[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t sl = s_begin + (int64_t)i * L::CH + (e >> 1) * 8 + 2 * t + (e & 1);
+        kpos[e] = sl < s_end ? (RANGE ? (int32_t)sl : sidx[sl - s_begin]) : -1;
+      }
     // S = Q K^T with the shared head-dim permutation (see the header);
     // four independent accumulation chains
     float s4[4][4] = {};
@@ -243,7 +286,6 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
       s[0][e] = s4[0][e] + s4[2][e];
       s[1][e] = s4[1][e] + s4[3][e];
     }
-    (void)qa;
     float x[2][4];
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -252,17 +294,16 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
       for (int e = 0; e < 4; ++e) {
         const int key = nt * 8 + 2 * t + (e & 1);
         float v = s[nt][e] * (p.scale_log2 * qscale_inv * sks[key]);
-        if (spos[key] < 0) v = -INFINITY;
+        if (kpos[nt * 2 + (e & 1)] < 0) v = -INFINITY;
         x[nt][e] = v;
         if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
       }
     if (RANGE) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        const int key = nt * 8 + 2 * t;
-        const int32_t pos = spos[key];
+        const int32_t pos = kpos[nt * 2];
         if (pos >= 0) {
-          const bool two = spos[key + 1] >= 0;
+          const bool two = kpos[nt * 2 + 1] >= 0;
           float* r0 = p.logits + ((int64_t)b * p.H + g) * p.logit_ld + pos;
           if (g < p.H) {
             if (two) *reinterpret_cast<float2*>(r0) = make_float2(x[nt][0], x[nt][1]);
@@ -336,9 +377,10 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
         }
       }
     }
-    __syncwarp();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
   }
-  cp_async_wait<0>();
 
   // ---- merge the warps into this CTA's partial (m, l, O) in shared memory
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -346,9 +388,9 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();
-  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NW warps] partials
-  float* mine = cmb + L::NW * (L::PART / 4);                    // merged partial of the CTA
-  {
+  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NC warps] partials
+  float* mine = cmb + L::NC * (L::PART / 4);                    // merged partial of the CTA
+  if (warp < L::NC) {
     float* wpart = cmb + warp * (L::PART / 4);
     if (t == 0) {
       wpart[g] = m0;
@@ -366,35 +408,39 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
       wpart[32 + (g + 8) * D + dcol + 2] = o[j][3];
     }
   }
+  // per-head merge factors of the warps, once: fac[w][h] = 2^(m_w - M_h)
+  __shared__ float fac[L::NC][16];
+  __shared__ float cfac[8][16];
+  __shared__ float cinv[16];
   __syncthreads();
-  for (int e = threadIdx.x; e < 16 * D; e += blockDim.x) {
-    const int h = e / D, c = e % D;
+  if (threadIdx.x < 16) {
+    const int h = threadIdx.x;
     float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < L::NW; ++w) M = fmaxf(M, cmb[w * (L::PART / 4) + h]);
-    float Ls = 0.f, Ov = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < L::NW; ++w) {
-        const float mw = cmb[w * (L::PART / 4) + h];
-        const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        Ls += cmb[w * (L::PART / 4) + 16 + h] * f;
-        Ov += cmb[w * (L::PART / 4) + 32 + h * D + c] * f;
-      }
+    for (int w = 0; w < L::NC; ++w) M = fmaxf(M, cmb[w * (L::PART / 4) + h]);
+    float Ls = 0.f;
+    for (int w = 0; w < L::NC; ++w) {
+      const float mw = cmb[w * (L::PART / 4) + h];
+      const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+      fac[w][h] = f;
+      Ls += cmb[w * (L::PART / 4) + 16 + h] * f;
     }
-    if (PARTIALS) {
-      float* part = p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D);
-      part[32 + h * D + c] = Ov;
-      if (c == 0) {
-        part[h] = M;
-        part[16 + h] = Ls;
+    float* dst = PARTIALS ? p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D) : mine;
+    dst[h] = M;
+    dst[16 + h] = Ls;
+  }
+  __syncthreads();
+  {
+    float* dst = PARTIALS ? p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D) : mine;
+    for (int e4 = threadIdx.x; e4 < 16 * D / 4; e4 += blockDim.x) {
+      const int h = (e4 * 4) / D;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < L::NC; ++w) {
+        const float4 v = reinterpret_cast<const float4*>(cmb + w * (L::PART / 4) + 32)[e4];
+        const float f = fac[w][h];
+        acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
       }
-    } else {
-      mine[32 + h * D + c] = Ov;
-      if (c == 0) {
-        mine[h] = M;
-        mine[16 + h] = Ls;
-      }
+      reinterpret_cast<float4*>(dst + 32)[e4] = acc;
     }
   }
   if (!PARTIALS) {
@@ -403,24 +449,39 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
     const int C = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
     cluster.sync();
-    const int hp = (16 + C - 1) / C;                 // heads merged by this CTA
-    const int h0 = r * hp, h1 = min(16, h0 + hp);
-    for (int e = threadIdx.x; e < (h1 - h0) * D; e += blockDim.x) {
-      const int h = h0 + e / D, c = e % D;
-      if (h >= p.H) continue;
+    if (threadIdx.x < 16) {
+      const int h = threadIdx.x;
       float M = -INFINITY;
       for (int q = 0; q < C; ++q) M = fmaxf(M, cluster.map_shared_rank(mine, q)[h]);
-      float Ls = 0.f, Ov = 0.f;
-      if (M != -INFINITY) {
-        for (int q = 0; q < C; ++q) {
-          const float* pq = cluster.map_shared_rank(mine, q);
-          const float mq = pq[h];
-          const float f = (mq == -INFINITY) ? 0.f : fast_exp2(mq - M);
-          Ls += pq[16 + h] * f;
-          Ov += pq[32 + h * D + c] * f;
-        }
+      float Ls = 0.f;
+      for (int q = 0; q < C; ++q) {
+        const float* pq = cluster.map_shared_rank(mine, q);
+        const float f = (M == -INFINITY || pq[h] == -INFINITY) ? 0.f : fast_exp2(pq[h] - M);
+        cfac[q][h] = f;
+        Ls += pq[16 + h] * f;
       }
-      p.O[((int64_t)b * p.H + h) * D + c] = __float2bfloat16_rn(Ls > 0.f ? Ov / Ls : 0.f);
+      cinv[h] = Ls > 0.f ? 1.f / Ls : 0.f;
+    }
+    __syncthreads();
+    const int hp = (16 + C - 1) / C;                 // heads merged by this CTA
+    const int h0 = r * hp, h1 = min(min(16, h0 + hp), p.H);
+    const int n4 = h1 > h0 ? (h1 - h0) * D / 4 : 0;
+    for (int e4 = threadIdx.x; e4 < n4; e4 += blockDim.x) {
+      const int h = h0 + (e4 * 4) / D;
+      const int off4 = (h0 * D) / 4 + e4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < C; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(cluster.map_shared_rank(mine, q) + 32)[off4];
+        const float f = cfac[q][h];
+        acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+      }
+      const float inv = cinv[h];
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(p.O + ((int64_t)b * p.H) * D + (int64_t)off4 * 4) = pk;
     }
     cluster.sync();                                    // peers read our partial until here
   }

@@ -210,7 +210,7 @@ template <int D>
 hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
                           cudaStream_t st) {
   prof_begin(st);
-  attn16_combine_kernel<D><<<items, 256, 0, st>>>(part, splits, H, O, ml);
+  attn16_combine_kernel<D><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml);
   return after_launch("attn16_combine_kernel", st);
 }
 
@@ -225,22 +225,26 @@ hs2_status launch_sparse_prefill(const Attn16Params& p, int grid, cudaStream_t s
 
 template <int D>
 hs2_status launch_decode_parts(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
-  hs2_status s = set_smem(decode_attn_kernel<D, false, true>, DecLayout<D>::SMEM);
+  using L = DecLayout<D>;
+  auto k = decode_attn_kernel<D, false, true>;
+  hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
   prof_begin(st);
-  decode_attn_kernel<D, false, true><<<batch * p.splits, DecLayout<D>::NW * 32, DecLayout<D>::SMEM, st>>>(p, ctx);
+  k<<<batch * p.splits, L::NT, L::SMEM, st>>>(p, ctx);
   return after_launch("decode_attn_kernel", st);
 }
 
 // One thread-block cluster of p.splits CTAs per sequence.
 template <int D>
 hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
-  hs2_status s = set_smem(decode_attn_kernel<D, false, false>, DecLayout<D>::SMEM);
+  using L = DecLayout<D>;
+  auto k = decode_attn_kernel<D, false, false>;
+  hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(batch * p.splits));
-  cfg.blockDim = dim3(DecLayout<D>::NW * 32);
-  cfg.dynamicSmemBytes = DecLayout<D>::SMEM;
+  cfg.blockDim = dim3(L::NT);
+  cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -250,7 +254,7 @@ hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<D, false, false>, p, ctx);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, p, ctx);
   if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_attn_kernel)");
   return after_launch("decode_attn_kernel", st);
 }
@@ -345,10 +349,12 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   p.part = part;
   p.logits = logits;
   p.logit_ld = w.ld;
-  hs2_status s = set_smem(decode_attn_kernel<D, true, true>, DecLayout<D>::SMEM);
+  using L = DecLayout<D>;
+  auto k = decode_attn_kernel<D, true, true>;
+  hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
   prof_begin(st);
-  decode_attn_kernel<D, true, true><<<batch * w.splits, DecLayout<D>::NW * 32, DecLayout<D>::SMEM, st>>>(p, ctx);
+  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx);
   if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
   if ((s = launch_combine<D>(part, w.splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
