@@ -276,19 +276,24 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
     krem -= above;
     lo = nlo;
     hi = nhi;
-    if (!cached && !listed && k - krem + in_range <= (uint32_t)TK_CAP) {
-      // long row: keep only the elements >= lo (all that can still be chosen)
+    if (!listed && k - krem + in_range <= (uint32_t)TK_CAP) {
+      // keep only the elements >= lo (all that can still be chosen): the next
+      // passes and the marking then touch about k elements, not the row
       if (threadIdx.x == 0) ncand = 0;
       __syncthreads();
       const uint32_t clo = lo;
-      tk_stream(src, n, [&](int64_t i, uint32_t raw) {
-        const uint32_t u = tk_clean(raw, ctx);
+      auto take = [&](int64_t i, uint32_t u) {
         if (u >= clo) {               // at most TK_CAP of them (counted above)
           const uint32_t slot = atomicAdd(&ncand, 1u);
           cval[slot] = u;
           cpos[slot] = (int32_t)i;
         }
-      });
+      };
+      if (cached) {
+        for (int64_t i = threadIdx.x; i < n; i += TK_THREADS) take(i, cache[i]);
+      } else {
+        tk_stream(src, n, [&](int64_t i, uint32_t raw) { take(i, tk_clean(raw, ctx)); });
+      }
       __syncthreads();
       listed = true;
     }
@@ -297,8 +302,8 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
   const uint32_t need_eq = krem;  // how many keys equal to T are taken
   const uint32_t eq_count = in_range;
 
-  // ---- mark and emit in position order
-  uint32_t* bm = cached ? small_bm : cache;
+  // ---- mark and emit in position order (a listed row no longer needs the cache)
+  uint32_t* bm = (cached && !listed) ? small_bm : cache;
   const int64_t words = (n + 31) >> 5;
   if (threadIdx.x == 0) pstar = INT64_MAX;
   if (listed) {
