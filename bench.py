@@ -502,10 +502,13 @@ def main():
     ap.add_argument("--T", type=int, default=None, help="override the prefill length (small profiling cases)")
     ap.add_argument("--decode-N", type=int, default=None, help="override the decode context (small profiling cases)")
     ap.add_argument("--only-decode", action="store_true", help="run the decode measurement only")
+    ap.add_argument("--decode-B", type=int, default=None, help="override the decode batch (small profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     if args.decode_N:
         DECODE["N"] = args.decode_N
+    if args.decode_B:
+        DECODE["B"] = args.decode_B
     if args.T:
         WORKLOAD["T"] = args.T
         WORKLOAD["n_needles"] = min(WORKLOAD["n_needles"], max(0, args.T // 512))

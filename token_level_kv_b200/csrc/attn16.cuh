@@ -71,39 +71,57 @@ __device__ __forceinline__ uint32_t swz_off(int row, int unit) {
   return (uint32_t)(row * D * 2 + ((unit ^ (row & 7)) << 4));
 }
 
-// Sparse prefill layer (row a6) over the shared bf16 KV: one query row per
-// warp (16 heads = the M of mma.sync), so the 4 warps of a CTA never merge.
-// K and V of a 16-key chunk travel as separate 8 KB stages of a per-warp
-// 5-stage cp.async ring (K_c, V_c, K_c+1, ...), so a warp keeps up to 4
-// stages (2 chunks) in flight while it computes; rows are stored at a
-// 2*D + 16 byte stride, which keeps the ldmatrix loads of 8 rows on 8
-// different bank groups.  The reference max of the online softmax moves only
-// when a row's max grows by more than 2^8 (lazy rescale of O).
+// Sparse prefill layer (row a6) over the shared bf16 KV.  A PAIR of warps
+// owns one query row; warp half h holds dims [h*D/2, (h+1)*D/2) of Q, of the
+// gathered K and V rows and of O (16 heads = the M of mma.sync).  Per 16-key
+// chunk each warp forms the partial S over its half of d; the two partials
+// meet in shared memory (double-buffered, one pair barrier per chunk) and both
+// warps add them in the same order, so both hold the same S and run the same
+// online softmax, and each adds P V for its half of d.  Halving O (64 fp32
+// registers a thread) puts 8 warps on an SM where one warp per row fitted 4,
+// which is what hides the gather and mma latencies.  K and V half rows of a
+// chunk travel as separate stages of a per-warp 5-stage cp.async ring
+// (K_c, V_c, K_c+1, ...), up to 4 stages in flight; rows are stored at a
+// D + 16 byte stride, which keeps the ldmatrix loads of 8 rows on 8 different
+// bank groups.  The reference max of the online softmax moves only when a
+// row's max grows by more than 2^8 (lazy rescale of O).
 template <int D>
 struct SpfLayout {
   static constexpr int CH = 16;
-  static constexpr int NST = 5;                    // stages per warp (K or V of one chunk)
-  static constexpr int ROW = 2 * D + 16;
+  static constexpr int HD = D / 2;                 // dims per warp
+  static constexpr int NST = 5;                    // stages per warp (K or V half rows of one chunk)
+  static constexpr int NPAIR = 4;                  // query rows in flight per CTA
+  static constexpr int NT = NPAIR * 64;
+  static constexpr int ROW = 2 * HD + 16;          // half row + pad
   static constexpr int STAGE = CH * ROW + CH * 4;  // rows + positions
-  static constexpr int Q_BYTES = 16 * D * 2;       // swizzled, per warp
+  static constexpr int Q_BYTES = 16 * HD * 2;      // swizzled half of Q, per warp
   static constexpr int WARP = NST * STAGE + Q_BYTES;
-  static constexpr size_t SMEM = 4 * (size_t)WARP + 128;
+  static constexpr int XCH = 2 * 2 * 32 * 8 * 4;   // per pair: [chunk parity][half][8 floats x 32 lanes]
+  static constexpr size_t SMEM = 2 * NPAIR * (size_t)WARP + NPAIR * (size_t)XCH;
 };
 
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(SpfLayout<D>::NT, 1)
 sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
   using L = SpfLayout<D>;
+  constexpr int HD = L::HD;
   extern __shared__ __align__(128) uint8_t smem_spf[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = warp >> 1, h = warp & 1;
   const int g = lane >> 2, t = lane & 3;
   uint8_t* wb = smem_spf + warp * L::WARP;
   uint8_t* sQ = wb + L::NST * L::STAGE;
   const uint32_t qa = smem_u32(sQ);
+  float4* xch = reinterpret_cast<float4*>(smem_spf + 2 * L::NPAIR * L::WARP + pair * L::XCH);
   const int cpi = (p.n_idx + L::CH - 1) / L::CH;
   const int64_t n_rows = p.n_rows;
+  const int dcol0 = h * HD;                          // this warp's first dim
+  // Q half row r, 16-byte unit u stored at unit u ^ (r & 7)
+  auto qoff = [](int r, int u) -> uint32_t { return (uint32_t)(r * HD * 2 + ((u ^ (r & 7)) << 4)); };
+  auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory"); };
+  int xc = 0;                                        // chunks so far (exchange buffer parity)
 
-  for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < n_rows; row += (int64_t)gridDim.x * 4) {
+  for (int64_t row = (int64_t)blockIdx.x * L::NPAIR + pair; row < n_rows; row += (int64_t)gridDim.x * L::NPAIR) {
     const int32_t* irow = p.idx + row * p.n_idx;
     // positions of a chunk (lanes 0-15, lanes 16-31 mirror them), loaded two
     // chunks before their stages are issued so the load latency is hidden
@@ -111,17 +129,17 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       const int sl = c * L::CH + (lane & 15);
       return (c < cpi && sl < p.n_idx) ? irow[sl] : -1;
     };
-    // stage sequence: 2c = K rows of chunk c, 2c + 1 = V rows of chunk c
+    // stage sequence: 2c = K half rows of chunk c, 2c + 1 = V half rows
     auto issue = [&](int sidx, int32_t pos) {
       const bool is_v = sidx & 1;
       uint8_t* st = wb + (sidx % L::NST) * L::STAGE;
       if (pos < -1 || pos >= p.kv_len) {
-        if (!is_v && lane < 16) report(ctx, ST_DEVICE_CHECK);
+        if (!is_v && h == 0 && lane < 16) report(ctx, ST_DEVICE_CHECK);
         pos = -1;
       }
       if (lane < 16) reinterpret_cast<int32_t*>(st + L::CH * L::ROW)[lane] = pos;
-      const uint8_t* base = reinterpret_cast<const uint8_t*>(is_v ? p.V : p.K);
-      constexpr int UPR = 2 * D / 16;
+      const uint8_t* base = reinterpret_cast<const uint8_t*>(is_v ? p.V : p.K) + dcol0 * 2;
+      constexpr int UPR = 2 * HD / 16;
 #pragma unroll
       for (int seg = lane; seg < L::CH * UPR; seg += 32) {
         const int i = seg / UPR, u = seg % UPR;
@@ -143,22 +161,22 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       cp_async_commit();
     }
     int32_t q1 = ldpos(2), q2 = ldpos(3);
-    // Q of the row (rows >= H are zero)
+    // this warp's half of Q (rows >= H are zero)
     {
-      const __nv_bfloat16* q = p.Q + row * p.H * D;
-      for (int u = lane; u < 16 * D / 8; u += 32) {
-        const int r = u / (D / 8), un = u % (D / 8);
+      const __nv_bfloat16* q = p.Q + row * p.H * D + dcol0;
+      for (int u = lane; u < 16 * HD / 8; u += 32) {
+        const int r = u / (HD / 8), un = u % (HD / 8);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (r < p.H) v = *reinterpret_cast<const uint4*>(q + r * D + un * 8);
-        *reinterpret_cast<uint4*>(sQ + swz_off<D>(r, un)) = v;
+        *reinterpret_cast<uint4*>(sQ + qoff(r, un)) = v;
       }
     }
-    float o[D / 8][4];
+    float o[HD / 8][4];
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    for (int c = 0; c < cpi; ++c) {
+    for (int c = 0; c < cpi; ++c, ++xc) {
       // K stage of chunk c: 2c; keep NST-1 stages issued ahead
       {
         const int nxt = 2 * c + L::NST - 1;           // K stage of chunk c + 2
@@ -170,14 +188,14 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       const uint8_t* ks = wb + ((2 * c) % L::NST) * L::STAGE;
       const int32_t* spos = reinterpret_cast<const int32_t*>(ks + L::CH * L::ROW);
       const uint32_t ka = smem_u32(ks);
-      // four independent accumulation chains (2 key tiles x 2 halves of d)
+      // partial S over this warp's half of d: four independent chains
       float s4[4][4] = {};
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < HD / 16; ++kk) {
         uint32_t a[4], b[4];
         {
           const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(a, qa + swz_off<D>(r, kk * 2 + (lane >> 4)));
+          ldsm_x4(a, qa + qoff(r, kk * 2 + (lane >> 4)));
         }
         {
           const int key = (lane & 7) + (lane >> 4) * 8;
@@ -186,11 +204,24 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
         mma_bf16_16816(s4[(kk & 1) * 2 + 0], a, b[0], b[1]);
         mma_bf16_16816(s4[(kk & 1) * 2 + 1], a, b[2], b[3]);
       }
+      // exchange the partials; S = S_half0 + S_half1 in both warps
       float s[2][4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        s[0][e] = s4[0][e] + s4[2][e];
-        s[1][e] = s4[1][e] + s4[3][e];
+      {
+        float4* mine = xch + ((xc & 1) * 2 + h) * 64;
+        const float4* other = xch + ((xc & 1) * 2 + (h ^ 1)) * 64;
+        const float4 w0 = make_float4(s4[0][0] + s4[2][0], s4[0][1] + s4[2][1], s4[0][2] + s4[2][2], s4[0][3] + s4[2][3]);
+        const float4 w1 = make_float4(s4[1][0] + s4[3][0], s4[1][1] + s4[3][1], s4[1][2] + s4[3][2], s4[1][3] + s4[3][3]);
+        mine[lane] = w0;
+        mine[32 + lane] = w1;
+        pair_sync();
+        const float4 v0 = other[lane], v1 = other[32 + lane];
+        if (h == 0) {
+          s[0][0] = w0.x + v0.x; s[0][1] = w0.y + v0.y; s[0][2] = w0.z + v0.z; s[0][3] = w0.w + v0.w;
+          s[1][0] = w1.x + v1.x; s[1][1] = w1.y + v1.y; s[1][2] = w1.z + v1.z; s[1][3] = w1.w + v1.w;
+        } else {
+          s[0][0] = v0.x + w0.x; s[0][1] = v0.y + w0.y; s[0][2] = v0.z + w0.z; s[0][3] = v0.w + w0.w;
+          s[1][0] = v1.x + w1.x; s[1][1] = v1.y + w1.y; s[1][2] = v1.z + w1.z; s[1][3] = v1.w + w1.w;
+        }
       }
       float x[2][4];
       float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -241,7 +272,7 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       l1 = l1 * al1 + ls1;
       if (al0 != 1.f || al1 != 1.f) {
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
+        for (int i = 0; i < HD / 8; ++i) {
           o[i][0] *= al0; o[i][1] *= al0;
           o[i][2] *= al1; o[i][3] *= al1;
         }
@@ -256,7 +287,7 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       __syncwarp();
       const uint32_t va = smem_u32(wb + ((2 * c + 1) % L::NST) * L::STAGE);
 #pragma unroll
-      for (int nd = 0; nd < D / 16; ++nd) {
+      for (int nd = 0; nd < HD / 16; ++nd) {
         uint32_t b[4];
         const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
         ldsm_x4_t(b, va + key * L::ROW + (nd * 2 + (lane >> 4)) * 16);
@@ -272,9 +303,9 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-    __nv_bfloat16* out = p.O + row * p.H * D;
+    __nv_bfloat16* out = p.O + row * p.H * D + dcol0;
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
+    for (int i = 0; i < HD / 8; ++i) {
       const int col = i * 8 + 2 * t;
       if (g < p.H) *reinterpret_cast<uint32_t*>(out + g * D + col) = pack_bf16x2(o[i][0] * i0, o[i][1] * i0);
       if (g + 8 < p.H)

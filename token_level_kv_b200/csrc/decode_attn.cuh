@@ -8,13 +8,18 @@
 // Key j of sequence b is E4M3(K[b,j,:]) * k_scale[b,j], likewise V.
 //
 // Design (sm_100a), HBM-bound: everything serves bytes in flight.
-//   * One producer warp streams 16-key chunks into a shared ring of NS stages
-//     (cp.async, completion tracked by cp.async.mbarrier.arrive on the stage's
-//     mbarrier), so almost the whole ring is in flight whatever the consumers
-//     are doing; NC consumer warps take chunk i from stage i % NS (consumer
-//     i % NC) and hand the stage back through its empty barrier.  Raw FP8
-//     rows sit at a padded stride so the fragment loads below are
-//     bank-conflict free.
+//   * One producer warp streams 16-key chunks into a shared ring of NS stages,
+//     so almost the whole ring is in flight whatever the consumers are doing;
+//     NC consumer warps take chunk i from stage i % NS (consumer i % NC) and
+//     hand the stage back through its empty barrier.  A range (a7) is
+//     contiguous in the cache: one elected lane moves each chunk's K and V
+//     with 3-D TMA tiles (box 128 bytes x 16 keys, 128-byte swizzle; keys past
+//     kv_len arrive as zeros), which keeps the whole copy off the load/store
+//     pipe.  A gather (a8) copies one row per lane pair with cp.async into
+//     rows padded to D + 16 bytes.  Both layouts make the fragment loads below
+//     bank-conflict free; the per-key scales always come by cp.async, and
+//     completion is tracked on the stage's mbarrier (transaction bytes plus
+//     cp.async.mbarrier.arrive).
 //   * The products run on mma.sync m16n8k16 in f16 with fp32 accumulation
 //     (the heads are M): every E4M3 code is an f16, so one cvt.rn.f16x2.e4m3x2
 //     widens two codes exactly.  Q enters in f16 after an exact power-of-two
@@ -59,29 +64,39 @@ namespace hs2 {
 
 namespace cg = cooperative_groups;
 
-template <int D>
+template <int D, bool RANGE>
 struct DecLayout {
-  static constexpr int NC = 7;                      // consumer warps (8 warps with the producer)
-  static constexpr int NT = (NC + 1) * 32;          // + one producer warp
-  static constexpr int NS = 20;                     // ring stages (16 keys each)
-  static constexpr int CH = 16;
-  static constexpr int KROW = D + 16;               // padded raw K row
-  static constexpr int VROW = D + 16;               // padded raw V row (conflict-free ldmatrix)
+  static constexpr int NP = 5;                      // consumer warp pairs
+  static constexpr int NC = 2 * NP;                 // consumer warps
+  static constexpr int HD = D / 2;                  // dims per consumer warp
+  static constexpr int NT = (NC + 1) * 32;          // + one producer warp (11 warps: <= 168 registers)
+  static constexpr int NS = 10;                     // ring stages (32 keys each)
+  static constexpr int CH = 32;
+  // gather stage: K rows, V rows at a padded stride, then the two scale rows
+  static constexpr int KROW = RANGE ? 128 : D + 16;
+  static constexpr int VROW = D + 16;
+  static constexpr int BOX = CH * 128;              // range stage: one TMA box, 128 bytes x 32 keys
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + CH * KROW;
-  static constexpr int OFF_KS = OFF_V + CH * VROW;
-  static constexpr int OFF_VS = OFF_KS + CH * 4;
-  static constexpr int STAGE = OFF_VS + CH * 4;
-  static constexpr int QROW = 2 * D + 16;           // padded f16 Q row
+  static constexpr int OFF_V = RANGE ? CH * D : CH * KROW;
+  static constexpr int STAGE = RANGE ? 2 * CH * D : 2 * CH * (D + 16) + 2 * CH * 4;
+  static constexpr int QROW = 2 * D + 32;           // padded f16 Q row (8-byte fragment loads conflict free)
   static constexpr int Q_BYTES = 16 * QROW;
   static constexpr int PART = (32 + 16 * D) * 4;    // one (m, l, O) partial
-  static constexpr int OFF_RING = Q_BYTES;
+  static constexpr int OFF_RING = (Q_BYTES + 1023) / 1024 * 1024;   // swizzled TMA boxes want 1 KB
+  static constexpr int OFF_SC = OFF_RING + NS * STAGE;              // range: scales [NS][2][CH]
   static constexpr int IDX = 2048 * 4;              // the CTA's index slice
-  static constexpr int OFF_IDX = OFF_RING + NS * STAGE;
-  static constexpr int OFF_BAR = OFF_IDX + IDX;
+  static constexpr int OFF_IDX = OFF_SC + (RANGE ? NS * 2 * CH * 4 : 0);
+  static constexpr int XCH = 2 * 2 * 32 * 8 * 4 + 16;   // per pair: [chunk parity][half][8 floats x 32 lanes] + flags
+  static constexpr int OFF_XCH = OFF_IDX + (RANGE ? 0 : IDX);
+  static constexpr int OFF_BAR = OFF_XCH + NP * XCH;
   static constexpr int MAIN = OFF_BAR + 2 * NS * 8;
-  static constexpr int MERGE = Q_BYTES + NC * PART + PART;
-  static constexpr size_t SMEM = (MAIN > MERGE ? MAIN : MERGE) + 128;
+  static constexpr int MERGE = Q_BYTES + NP * PART + PART;
+  static constexpr size_t SMEM = (MAIN > MERGE ? MAIN : MERGE) + 1024;   // + base alignment
+  // scale rows of stage s
+  __device__ static float* kscale(uint8_t* smem, int s) {
+    return RANGE ? reinterpret_cast<float*>(smem + OFF_SC) + s * 2 * CH
+                 : reinterpret_cast<float*>(smem + OFF_RING + s * STAGE + 2 * CH * (D + 16));
+  }
 };
 
 struct DecParams {
@@ -104,12 +119,15 @@ struct DecParams {
   int64_t logit_ld;
 };
 
+// tmK / tmV: 3-D maps {D, kv_len, batch} over the codes (range only; a gather
+// passes unused maps).
 template <int D, bool RANGE, bool PARTIALS>
-__global__ void __launch_bounds__(DecLayout<D>::NT, 1)
-decode_attn_kernel(DecParams p, DevCtx ctx) {
-  using L = DecLayout<D>;
+__global__ void __launch_bounds__(DecLayout<D, RANGE>::NT, 1)
+decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV) {
+  using L = DecLayout<D, RANGE>;
   extern __shared__ __align__(128) uint8_t smem_dec[];
-  uint8_t* smem = smem_dec;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dec) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int b = blockIdx.x / p.splits;
@@ -127,8 +145,8 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::NS; ++s) {
-      mbar_init(&full[s], 32);             // the producer lanes' cp.async arrivals
-      mbar_init(&empty[s], 1);             // the consuming warp
+      mbar_init(&full[s], RANGE ? 33 : 32);  // the producer lanes' cp.async arrivals (+ the TMA lane)
+      mbar_init(&empty[s], 2);             // the consuming warp pair
     }
     fence_barrier_init();
   }
@@ -180,38 +198,68 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
   // chunk i -> stage i % NS; the first ring round needs no empty wait, so it
   // is issued before the block-wide barrier below (nothing can block there)
   constexpr int UPR = D / 16;                        // 16-byte units per FP8 row
-  const int pkey = lane >> 1, pu0 = (lane & 1) * (UPR / 2);
+  constexpr int RPI = 32 / UPR;                      // rows per copy instruction (gather)
   auto produce = [&](int i) -> bool {
     const int s = i % L::NS;
     if (!mbar_wait(&empty[s], (uint32_t)(((i / L::NS) & 1) ^ 1), ctx)) return false;
     uint8_t* st = ring + s * L::STAGE;
-    const int64_t sl = s_begin + (int64_t)i * L::CH + pkey;
-    const int32_t pk = sl < s_end ? (RANGE ? (int32_t)sl : sidx[sl - s_begin]) : -1;
-    const int64_t row = seq + (pk < 0 ? 0 : pk);
-    const uint8_t* ksrc = p.K + row * D + pu0 * 16;
-    const uint8_t* vsrc = p.V + row * D + pu0 * 16;
-    const uint32_t kdst = smem_u32(st + L::OFF_K + pkey * L::KROW + pu0 * 16);
-    const uint32_t vdst = smem_u32(st + L::OFF_V + pkey * L::VROW + pu0 * 16);
+    if (RANGE) {
+      const int64_t pos0 = s_begin + (int64_t)i * L::CH;
+      if (lane == 0) {
+        mbar_expect_tx(&full[s], 2 * L::CH * D);
 #pragma unroll
-    for (int u = 0; u < UPR / 2; ++u) {
-      cp_async16(kdst + u * 16, ksrc + u * 16, pk >= 0);
-      cp_async16(vdst + u * 16, vsrc + u * 16, pk >= 0);
+        for (int bx = 0; bx < D / 128; ++bx) {
+          tma_load_3d(st + L::OFF_K + bx * L::BOX, &tmK, &full[s], bx * 128, (int)pos0, b);
+          tma_load_3d(st + L::OFF_V + bx * L::BOX, &tmV, &full[s], bx * 128, (int)pos0, b);
+        }
+      }
+      float* sc = L::kscale(smem, s);
+      if (lane < L::CH) {
+        const bool ok = pos0 + lane < s_end;
+        const int64_t row = seq + (ok ? pos0 + lane : 0);
+        cp_async4(smem_u32(sc + lane), p.ks + row, ok);
+        cp_async4(smem_u32(sc + L::CH + lane), p.vs + row, ok);
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+      return true;
     }
-    if ((lane & 1) == 0) {
-      cp_async4(smem_u32(st + L::OFF_KS + pkey * 4), p.ks + row, pk >= 0);
-      cp_async4(smem_u32(st + L::OFF_VS + pkey * 4), p.vs + row, pk >= 0);
+    // lane j holds the position of stage row j; each copy instruction moves
+    // RPI whole rows (consecutive lanes, consecutive 16-byte units)
+    const int64_t sl = s_begin + (int64_t)i * L::CH + lane;
+    const int32_t pk = sl < s_end ? sidx[sl - s_begin] : -1;
+    {
+      const int64_t row = seq + (pk < 0 ? 0 : pk);
+      float* sc = L::kscale(smem, s);
+      cp_async4(smem_u32(sc + lane), p.ks + row, pk >= 0);
+      cp_async4(smem_u32(sc + L::CH + lane), p.vs + row, pk >= 0);
+    }
+    const int ur = lane / UPR, uu = lane % UPR;
+#pragma unroll 4
+    for (int j = 0; j < L::CH / RPI; ++j) {
+      const int r = j * RPI + ur;
+      const int32_t pr_ = __shfl_sync(0xffffffffu, pk, r);
+      const int64_t row = seq + (pr_ < 0 ? 0 : pr_);
+      cp_async16(smem_u32(st + L::OFF_K + r * L::KROW + uu * 16), p.K + row * D + uu * 16, pr_ >= 0);
+      cp_async16(smem_u32(st + L::OFF_V + r * L::VROW + uu * 16), p.V + row * D + uu * 16, pr_ >= 0);
     }
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
     return true;
   };
   const int first_round = min(n_chunks, L::NS);
   bool prod_ok = true;
-  if (warp == L::NC)
-    for (int i = 0; i < first_round && prod_ok; ++i) prod_ok = produce(i);
+  int issued = 0;
+  if (warp == L::NC) {
+    if (RANGE && lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    while (issued < first_round && prod_ok)
+      if ((prod_ok = produce(issued))) ++issued;
+  }
 
-  float o[D / 8][4];
+  float o[L::HD / 8][4];
 #pragma unroll
-  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  for (int i = 0; i < L::HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float qscale_inv = 1.f;
   // ---- Q -> f16 with an exact power-of-two prescale (largest element in
@@ -243,182 +291,225 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
   __syncthreads();                                   // Q in shared memory
 
   if (warp == L::NC) {
-    for (int i = first_round; i < n_chunks && prod_ok; ++i) prod_ok = produce(i);
+    while (issued < n_chunks && prod_ok)
+      if ((prod_ok = produce(issued))) ++issued;
     asm volatile("cp.async.wait_all;" ::: "memory");  // every issued copy lands before the merge reuses the ring
+    if (RANGE && lane == 0)                           // and every TMA tile (already done unless a wait gave up)
+      for (int i = max(0, issued - L::NS); i < issued; ++i) mbar_drain(&full[i % L::NS], (uint32_t)((i / L::NS) & 1));
   } else {
     // ------------------------------------------------------------ consumers
-    for (int i = warp; i < n_chunks; i += L::NC) {
+    // pair `pr` takes steps i = pr, pr + NP, ... of 32 keys.  Warp half `hf`
+    // forms S over the whole head dim for keys [16*hf, 16*hf + 16) of the
+    // stage; the two halves of S meet in shared memory, both warps run the
+    // same online softmax over the 32 keys and each adds P V for dims
+    // [hf*HD, (hf+1)*HD) of O.
+    const int pr = warp >> 1, hf = warp & 1;
+    float4* xch = reinterpret_cast<float4*>(smem + L::OFF_XCH + pr * L::XCH);
+    volatile int* xok = reinterpret_cast<volatile int*>(xch + 4 * 64);   // [step parity][half]
+    int xc = 0;
+    for (int i = pr; i < n_chunks; i += L::NP, ++xc) {
       const int slot = i % L::NS;
-      if (!mbar_wait(&full[slot], (uint32_t)((i / L::NS) & 1), ctx)) break;
+      bool both_ok;
+      // both warps of the pair reach the pair barrier below on every step and
+      // leave the loop together: a timed-out wait still takes part in the
+      // exchange (its S is junk) and both warps then see the failure
+      const bool ok = mbar_wait(&full[slot], (uint32_t)((i / L::NS) & 1), ctx);
       const uint8_t* st = ring + slot * L::STAGE;
-      const float* sks = reinterpret_cast<const float*>(st + L::OFF_KS);
-      const float* svs = reinterpret_cast<const float*>(st + L::OFF_VS);
-      // positions of this thread's keys 2t, 2t+1, 8+2t, 9+2t (-1: empty slot)
-      int32_t kpos[4];
+      const float* sks = L::kscale(smem, slot);
+      const float* svs = sks + L::CH;
+      const int64_t sl0 = s_begin + (int64_t)i * L::CH;
+      // S = Q K^T for this warp's 16 keys with the shared head-dim permutation
+      // (see the header); four independent accumulation chains
+      float s4[4][4] = {};
+      const uint8_t* kraw = st + L::OFF_K;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int64_t sl = s_begin + (int64_t)i * L::CH + (e >> 1) * 8 + 2 * t + (e & 1);
-        kpos[e] = sl < s_end ? (RANGE ? (int32_t)sl : sidx[sl - s_begin]) : -1;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int d0 = kk * 16 + 4 * t;
+        uint32_t a[4];
+        {
+          const uint2 q0 = *reinterpret_cast<const uint2*>(sQ + g * L::QROW + d0 * 2);
+          const uint2 q1 = *reinterpret_cast<const uint2*>(sQ + (g + 8) * L::QROW + d0 * 2);
+          a[0] = q0.x; a[2] = q0.y; a[1] = q1.x; a[3] = q1.y;
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          // range: row r of box kk/8, 16-byte unit (kk%8) ^ (r%8) (128-byte swizzle)
+          const int r = 16 * hf + nt * 8 + g;
+          const int koff = RANGE ? (kk >> 3) * L::BOX + r * 128 + (((kk & 7) ^ g) << 4) + 4 * t
+                                 : r * L::KROW + d0;
+          const uint32_t kw = *reinterpret_cast<const uint32_t*>(kraw + koff);
+          mma_f16_16816(s4[(kk & 1) * 2 + nt], a, e4m3x2_to_f16x2((uint16_t)(kw & 0xffffu)),
+                        e4m3x2_to_f16x2((uint16_t)(kw >> 16)));
+        }
       }
-    // S = Q K^T with the shared head-dim permutation (see the header);
-    // four independent accumulation chains
-    float s4[4][4] = {};
-    const uint8_t* kraw = st + L::OFF_K;
-#pragma unroll 4
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int d0 = kk * 16 + 4 * t;
-      uint32_t a[4];
+      // n-tiles 0, 1: keys 0-15 (warp 0's); 2, 3: keys 16-31 (warp 1's)
+      float s[4][4];
       {
-        const uint2 q0 = *reinterpret_cast<const uint2*>(sQ + g * L::QROW + d0 * 2);
-        const uint2 q1 = *reinterpret_cast<const uint2*>(sQ + (g + 8) * L::QROW + d0 * 2);
-        a[0] = q0.x; a[2] = q0.y; a[1] = q1.x; a[3] = q1.y;
+        float4* mine = xch + ((xc & 1) * 2 + hf) * 64;
+        const float4* other = xch + ((xc & 1) * 2 + (hf ^ 1)) * 64;
+        const float4 w0 = make_float4(s4[0][0] + s4[2][0], s4[0][1] + s4[2][1], s4[0][2] + s4[2][2], s4[0][3] + s4[2][3]);
+        const float4 w1 = make_float4(s4[1][0] + s4[3][0], s4[1][1] + s4[3][1], s4[1][2] + s4[3][2], s4[1][3] + s4[3][3]);
+        mine[lane] = w0;
+        mine[32 + lane] = w1;
+        if (lane == 0) xok[(xc & 1) * 2 + hf] = ok ? 1 : 0;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
+        const float4 v0 = other[lane], v1 = other[32 + lane];
+        both_ok = ok && xok[(xc & 1) * 2 + (hf ^ 1)] != 0;
+        const float4 t0 = hf ? v0 : w0, t1 = hf ? v1 : w1, t2 = hf ? w0 : v0, t3 = hf ? w1 : v1;
+        s[0][0] = t0.x; s[0][1] = t0.y; s[0][2] = t0.z; s[0][3] = t0.w;
+        s[1][0] = t1.x; s[1][1] = t1.y; s[1][2] = t1.z; s[1][3] = t1.w;
+        s[2][0] = t2.x; s[2][1] = t2.y; s[2][2] = t2.z; s[2][3] = t2.w;
+        s[3][0] = t3.x; s[3][1] = t3.y; s[3][2] = t3.z; s[3][3] = t3.w;
       }
+      if (!both_ok) break;
+      // positions of this thread's keys 8*nt + 2t + e (-1: empty slot)
+      int32_t kpos[4][2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const uint32_t kw = *reinterpret_cast<const uint32_t*>(kraw + (nt * 8 + g) * L::KROW + d0);
-        mma_f16_16816(s4[(kk & 1) * 2 + nt], a, e4m3x2_to_f16x2((uint16_t)(kw & 0xffffu)),
-                      e4m3x2_to_f16x2((uint16_t)(kw >> 16)));
-      }
-    }
-    float s[2][4];
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s[0][e] = s4[0][e] + s4[2][e];
-      s[1][e] = s4[1][e] + s4[3][e];
-    }
-    float x[2][4];
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int e = 0; e < 2; ++e) {
+          const int64_t sl = sl0 + nt * 8 + 2 * t + e;
+          kpos[nt][e] = sl < s_end ? (RANGE ? (int32_t)sl : sidx[sl - s_begin]) : -1;
+        }
+      float x[4][4];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = nt * 8 + 2 * t + (e & 1);
-        float v = s[nt][e] * (p.scale_log2 * qscale_inv * sks[key]);
-        if (kpos[nt * 2 + (e & 1)] < 0) v = -INFINITY;
-        x[nt][e] = v;
-        if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
-      }
-    if (RANGE) {
+        for (int e = 0; e < 4; ++e) {
+          const int key = nt * 8 + 2 * t + (e & 1);
+          float v = s[nt][e] * (p.scale_log2 * qscale_inv * sks[key]);
+          if (kpos[nt][e & 1] < 0) v = -INFINITY;
+          x[nt][e] = v;
+          if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+        }
+      if (RANGE) {                                   // each warp writes the logits of its own keys
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int32_t pos = kpos[nt * 2];
-        if (pos >= 0) {
-          const bool two = kpos[nt * 2 + 1] >= 0;
-          float* r0 = p.logits + ((int64_t)b * p.H + g) * p.logit_ld + pos;
-          if (g < p.H) {
-            if (two) *reinterpret_cast<float2*>(r0) = make_float2(x[nt][0], x[nt][1]);
-            else r0[0] = x[nt][0];
-          }
-          if (g + 8 < p.H) {
-            float* r1 = r0 + 8 * p.logit_ld;
-            if (two) *reinterpret_cast<float2*>(r1) = make_float2(x[nt][2], x[nt][3]);
-            else r1[0] = x[nt][2];
+        for (int nt = 0; nt < 4; ++nt) {
+          const int32_t pos = kpos[nt][0];
+          if ((nt >> 1) == hf && pos >= 0) {
+            const bool two = kpos[nt][1] >= 0;
+            float* r0 = p.logits + ((int64_t)b * p.H + g) * p.logit_ld + pos;
+            if (g < p.H) {
+              if (two) *reinterpret_cast<float2*>(r0) = make_float2(x[nt][0], x[nt][1]);
+              else r0[0] = x[nt][0];
+            }
+            if (g + 8 < p.H) {
+              float* r1 = r0 + 8 * p.logit_ld;
+              if (two) *reinterpret_cast<float2*>(r1) = make_float2(x[nt][2], x[nt][3]);
+              else r1[0] = x[nt][2];
+            }
           }
         }
       }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    // lazy rescale: move the reference max only when it grows by > 2^8
-    float al0 = 1.f, al1 = 1.f;
-    if (mx0 > m0 + 8.f) {
-      al0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - mx0);
-      m0 = mx0;
-    }
-    if (mx1 > m1 + 8.f) {
-      al1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - mx1);
-      m1 = mx1;
-    }
-    const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
-    const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
-    float pr[2][4];
-    float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float pe = fast_exp2(x[nt][e] - (e < 2 ? mu0 : mu1));
-        if (e < 2) ls0 += pe; else ls1 += pe;
-        pr[nt][e] = pe * svs[nt * 8 + 2 * t + (e & 1)];
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      // lazy rescale: move the reference max only when it grows by > 2^8
+      float al0 = 1.f, al1 = 1.f;
+      if (mx0 > m0 + 8.f) {
+        al0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - mx0);
+        m0 = mx0;
       }
-    l0 = l0 * al0 + ls0;
-    l1 = l1 * al1 + ls1;
-    if (al0 != 1.f || al1 != 1.f) {
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        o[i][0] *= al0; o[i][1] *= al0;
-        o[i][2] *= al1; o[i][3] *= al1;
+      if (mx1 > m1 + 8.f) {
+        al1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - mx1);
+        m1 = mx1;
       }
-    }
-    uint32_t ap[4];
-    ap[0] = pack_f16x2(pr[0][0], pr[0][1]);
-    ap[1] = pack_f16x2(pr[0][2], pr[0][3]);
-    ap[2] = pack_f16x2(pr[1][0], pr[1][1]);
-    ap[3] = pack_f16x2(pr[1][2], pr[1][3]);
-    // O += P V, B fragments from the raw codes (see the header): per 32 bytes
-    // of d, 4 n-tiles j = 4*blk + 2*half + parity covering dims c0 + 2n + parity
-    {
+      const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
+      const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
+      float pv[4][4];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pe = fast_exp2(x[nt][e] - (e < 2 ? mu0 : mu1));
+          if (e < 2) ls0 += pe; else ls1 += pe;
+          pv[nt][e] = pe * svs[nt * 8 + 2 * t + (e & 1)];
+        }
+      l0 = l0 * al0 + ls0;
+      l1 = l1 * al1 + ls1;
+      if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+        for (int j = 0; j < L::HD / 8; ++j) {
+          o[j][0] *= al0; o[j][1] *= al0;
+          o[j][2] *= al1; o[j][3] *= al1;
+        }
+      }
+      // O += P V over this warp's half of d, in two k-steps of 16 keys; B
+      // fragments from the raw codes (see the header): per 32 bytes of d, 4
+      // n-tiles j = 4*blk + 2*half + parity covering dims c0 + 2n + parity
       const uint32_t va = smem_u32(st + L::OFF_V);
-      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int blk = 0; blk < D / 32; ++blk) {
-        uint32_t r[4];
-        ldsm_x4_t(r, va + key * L::VROW + blk * 32 + (lane >> 4) * 16);
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t ap[4];
+        ap[0] = pack_f16x2(pv[2 * ks][0], pv[2 * ks][1]);
+        ap[1] = pack_f16x2(pv[2 * ks][2], pv[2 * ks][3]);
+        ap[2] = pack_f16x2(pv[2 * ks + 1][0], pv[2 * ks + 1][1]);
+        ap[3] = pack_f16x2(pv[2 * ks + 1][2], pv[2 * ks + 1][3]);
+        const int key = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t px = __byte_perm(r[2 * half], r[2 * half + 1], 0x6420);
-          const uint32_t py = __byte_perm(r[2 * half], r[2 * half + 1], 0x7531);
-          mma_f16_16816(o[4 * blk + 2 * half], ap, e4m3x2_to_f16x2((uint16_t)(px & 0xffffu)),
-                        e4m3x2_to_f16x2((uint16_t)(px >> 16)));
-          mma_f16_16816(o[4 * blk + 2 * half + 1], ap, e4m3x2_to_f16x2((uint16_t)(py & 0xffffu)),
-                        e4m3x2_to_f16x2((uint16_t)(py >> 16)));
+        for (int b2 = 0; b2 < L::HD / 32; ++b2) {
+          const int blk = hf * (L::HD / 32) + b2;
+          uint32_t r[4];
+          const int vu = (blk & 3) * 2 + (lane >> 4);  // range: 16-byte unit within box blk/4
+          ldsm_x4_t(r, RANGE ? va + (blk >> 2) * L::BOX + key * 128 + ((vu ^ (lane & 7)) << 4)
+                             : va + key * L::VROW + blk * 32 + (lane >> 4) * 16);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t px = __byte_perm(r[2 * half], r[2 * half + 1], 0x6420);
+            const uint32_t py = __byte_perm(r[2 * half], r[2 * half + 1], 0x7531);
+            mma_f16_16816(o[4 * b2 + 2 * half], ap, e4m3x2_to_f16x2((uint16_t)(px & 0xffffu)),
+                          e4m3x2_to_f16x2((uint16_t)(px >> 16)));
+            mma_f16_16816(o[4 * b2 + 2 * half + 1], ap, e4m3x2_to_f16x2((uint16_t)(py & 0xffffu)),
+                          e4m3x2_to_f16x2((uint16_t)(py >> 16)));
+          }
         }
       }
-    }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
   }
 
-  // ---- merge the warps into this CTA's partial (m, l, O) in shared memory
+  // ---- merge the pairs into this CTA's partial (m, l, O) in shared memory
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();
-  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NC warps] partials
-  float* mine = cmb + L::NC * (L::PART / 4);                    // merged partial of the CTA
+  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NP pairs] partials
+  float* mine = cmb + L::NP * (L::PART / 4);                    // merged partial of the CTA
   if (warp < L::NC) {
-    float* wpart = cmb + warp * (L::PART / 4);
-    if (t == 0) {
+    const int pr = warp >> 1, hf = warp & 1;
+    float* wpart = cmb + pr * (L::PART / 4);
+    if (t == 0 && hf == 0) {
       wpart[g] = m0;
       wpart[g + 8] = m1;
       wpart[16 + g] = l0;
       wpart[16 + g + 8] = l1;
     }
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      // n-tile j: c0 = 16*(j/2), parity j&1; element e at n = 2t + (e&1)
-      const int dcol = 16 * (j >> 1) + 4 * t + (j & 1);
+    for (int j = 0; j < L::HD / 8; ++j) {
+      // local n-tile j: c0 = 16*(j/2), parity j&1; element e at n = 2t + (e&1)
+      const int dcol = hf * L::HD + 16 * (j >> 1) + 4 * t + (j & 1);
       wpart[32 + g * D + dcol] = o[j][0];
       wpart[32 + g * D + dcol + 2] = o[j][1];
       wpart[32 + (g + 8) * D + dcol] = o[j][2];
       wpart[32 + (g + 8) * D + dcol + 2] = o[j][3];
     }
   }
-  // per-head merge factors of the warps, once: fac[w][h] = 2^(m_w - M_h)
-  __shared__ float fac[L::NC][16];
+  // per-head merge factors of the pairs, once: fac[w][h] = 2^(m_w - M_h)
+  __shared__ float fac[L::NP][16];
   __shared__ float cfac[8][16];
   __shared__ float cinv[16];
   __syncthreads();
   if (threadIdx.x < 16) {
     const int h = threadIdx.x;
     float M = -INFINITY;
-    for (int w = 0; w < L::NC; ++w) M = fmaxf(M, cmb[w * (L::PART / 4) + h]);
+    for (int w = 0; w < L::NP; ++w) M = fmaxf(M, cmb[w * (L::PART / 4) + h]);
     float Ls = 0.f;
-    for (int w = 0; w < L::NC; ++w) {
+    for (int w = 0; w < L::NP; ++w) {
       const float mw = cmb[w * (L::PART / 4) + h];
       const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
       fac[w][h] = f;
@@ -435,7 +526,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx) {
       const int h = (e4 * 4) / D;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < L::NC; ++w) {
+      for (int w = 0; w < L::NP; ++w) {
         const float4 v = reinterpret_cast<const float4*>(cmb + w * (L::PART / 4) + 32)[e4];
         const float f = fac[w][h];
         acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;

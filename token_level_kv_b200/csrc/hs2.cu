@@ -117,6 +117,23 @@ hs2_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint6
   return HS2_OK;
 }
 
+// 3-D u8 tensor {inner, mid, outer} with byte strides (mid_stride, outer_stride),
+// 128-byte swizzle; out-of-range boxes read as zeros.
+hs2_status make_map_u8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                          uint64_t mid_stride, uint64_t outer_stride, uint32_t box_inner, uint32_t box_mid) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {mid_stride, outer_stride};
+  cuuint32_t box[3] = {box_inner, box_mid, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HS2_OK;
+}
+
 // ------------------------------------------------------------------ profiling
 constexpr int kMaxProf = 4096;
 struct ProfRec {
@@ -219,25 +236,26 @@ hs2_status launch_sparse_prefill(const Attn16Params& p, int grid, cudaStream_t s
   hs2_status s = set_smem(sparse_prefill_kernel<D>, SpfLayout<D>::SMEM);
   if (s != HS2_OK) return s;
   prof_begin(st);
-  sparse_prefill_kernel<D><<<grid, 128, SpfLayout<D>::SMEM, st>>>(p, ctx);
+  sparse_prefill_kernel<D><<<grid, SpfLayout<D>::NT, SpfLayout<D>::SMEM, st>>>(p, ctx);
   return after_launch("sparse_prefill_kernel", st);
 }
 
 template <int D>
 hs2_status launch_decode_parts(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
-  using L = DecLayout<D>;
+  using L = DecLayout<D, false>;
   auto k = decode_attn_kernel<D, false, true>;
   hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
+  const CUtensorMap unused{};
   prof_begin(st);
-  k<<<batch * p.splits, L::NT, L::SMEM, st>>>(p, ctx);
+  k<<<batch * p.splits, L::NT, L::SMEM, st>>>(p, ctx, unused, unused);
   return after_launch("decode_attn_kernel", st);
 }
 
 // One thread-block cluster of p.splits CTAs per sequence.
 template <int D>
 hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st, const DevCtx& ctx) {
-  using L = DecLayout<D>;
+  using L = DecLayout<D, false>;
   auto k = decode_attn_kernel<D, false, false>;
   hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
@@ -254,7 +272,8 @@ hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k, p, ctx);
+  const CUtensorMap unused{};
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, p, ctx, unused, unused);
   if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(decode_attn_kernel)");
   return after_launch("decode_attn_kernel", st);
 }
@@ -349,12 +368,19 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   p.part = part;
   p.logits = logits;
   p.logit_ld = w.ld;
-  using L = DecLayout<D>;
+  using L = DecLayout<D, true>;
   auto k = decode_attn_kernel<D, true, true>;
   hs2_status s = set_smem(k, L::SMEM);
   if (s != HS2_OK) return s;
+  CUtensorMap mK, mV;   // {D, kv_len, batch} codes; keys past kv_len read as zeros
+  if ((s = make_map_u8_3d(&mK, K, D, (uint64_t)kv_len, (uint64_t)batch, D, (uint64_t)kv_stride * D, 128,
+                          L::CH)) != HS2_OK)
+    return s;
+  if ((s = make_map_u8_3d(&mV, V, D, (uint64_t)kv_len, (uint64_t)batch, D, (uint64_t)kv_stride * D, 128,
+                          L::CH)) != HS2_OK)
+    return s;
   prof_begin(st);
-  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx);
+  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
   if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
   if ((s = launch_combine<D>(part, w.splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
@@ -533,7 +559,7 @@ hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int sms = 0;
   if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
-  const int grid = (int)std::min<int64_t>((Tq + 3) / 4, sms);
+  const int grid = (int)std::min<int64_t>((Tq + SpfLayout<256>::NPAIR - 1) / SpfLayout<256>::NPAIR, sms);
   return d == 256 ? launch_sparse_prefill<256>(p, grid, st, ctx) : launch_sparse_prefill<128>(p, grid, st, ctx);
 }
 
