@@ -112,6 +112,12 @@ class ClockSampler:
 # workload arithmetic
 # ---------------------------------------------------------------------------
 
+# DRAM bytes per query row of a launch, from one ncu capture of the kernel as
+# it stands (113.8 MB read + 39.5 MB written by one T = 8192 launch); set to
+# None whenever the kernel changes.
+DRAM_BYTES_PER_ROW = {"sparse_prefill_kernel": (113.825024e6 + 39.492096e6) / 8192}
+
+
 def prefill_flops(T, H, d, window, topk, n_sparse):
     full = 4.0 * d * H * T * (T + 1) / 2                       # QK^T and PV over the causal pairs
     n_idx = window + topk
@@ -322,8 +328,12 @@ def run_ours(args, rank, world, dist):
     roof = None
     if dom in work:
         ach = work[dom] / (kern[dom]["avg_ms"] * 1e-3) / 1e12
+        tr = DRAM_BYTES_PER_ROW.get(dom)
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "traffic": tr * T if tr is not None else None,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one T=8192 launch, "
+                                  "scaled by query rows (every term grows with T)" if tr is not None else None,
                 "peak_source": f"{peak_src} bf16_tflops (burst: kernels of a few ms, timed one by one)"}
     sel_ms = sum(kern.get(n, {"avg_ms": 0.0})["avg_ms"] for n in ("fa_fwd_kernel", "select_sigma_kernel",
                                                                   "topk_select_kernel"))

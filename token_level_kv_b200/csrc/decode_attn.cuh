@@ -82,6 +82,8 @@ struct DecLayout {
   static constexpr int QROW = 2 * D + 32;           // padded f16 Q row (8-byte fragment loads conflict free)
   static constexpr int Q_BYTES = 16 * QROW;
   static constexpr int PART = (32 + 16 * D) * 4;    // one (m, l, O) partial
+  static constexpr int PROW = D + 16;               // padded O row of a pair's partial (conflict-free float4 stores)
+  static constexpr int PPART = (32 + 16 * PROW) * 4;
   static constexpr int OFF_RING = (Q_BYTES + 1023) / 1024 * 1024;   // swizzled TMA boxes want 1 KB
   static constexpr int OFF_SC = OFF_RING + NS * STAGE;              // range: scales [NS][2][CH]
   static constexpr int IDX = 2048 * 4;              // the CTA's index slice
@@ -90,7 +92,7 @@ struct DecLayout {
   static constexpr int OFF_XCH = OFF_IDX + (RANGE ? 0 : IDX);
   static constexpr int OFF_BAR = OFF_XCH + NP * XCH;
   static constexpr int MAIN = OFF_BAR + 2 * NS * 8;
-  static constexpr int MERGE = Q_BYTES + NP * PART + PART;
+  static constexpr int MERGE = Q_BYTES + NP * PPART + PART;
   static constexpr size_t SMEM = (MAIN > MERGE ? MAIN : MERGE) + 1024;   // + base alignment
   // scale rows of stage s
   __device__ static float* kscale(uint8_t* smem, int s) {
@@ -478,25 +480,26 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();
-  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NP pairs] partials
-  float* mine = cmb + L::NP * (L::PART / 4);                    // merged partial of the CTA
+  float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NP pairs] partials, O rows padded
+  float* mine = cmb + L::NP * (L::PPART / 4);                   // merged partial of the CTA
   if (warp < L::NC) {
     const int pr = warp >> 1, hf = warp & 1;
-    float* wpart = cmb + pr * (L::PART / 4);
+    float* wpart = cmb + pr * (L::PPART / 4);
     if (t == 0 && hf == 0) {
       wpart[g] = m0;
       wpart[g + 8] = m1;
       wpart[16 + g] = l0;
       wpart[16 + g + 8] = l1;
     }
+    // n-tiles 2q and 2q+1 (q = 2*b2 + half) hold, for rows g and g+8, the four
+    // consecutive dims c0 + 4t .. c0 + 4t + 3 (c0 = hf*HD + 16q): one float4 each
 #pragma unroll
-    for (int j = 0; j < L::HD / 8; ++j) {
-      // local n-tile j: c0 = 16*(j/2), parity j&1; element e at n = 2t + (e&1)
-      const int dcol = hf * L::HD + 16 * (j >> 1) + 4 * t + (j & 1);
-      wpart[32 + g * D + dcol] = o[j][0];
-      wpart[32 + g * D + dcol + 2] = o[j][1];
-      wpart[32 + (g + 8) * D + dcol] = o[j][2];
-      wpart[32 + (g + 8) * D + dcol + 2] = o[j][3];
+    for (int q = 0; q < L::HD / 16; ++q) {
+      const int dcol = hf * L::HD + 16 * q + 4 * t;
+      *reinterpret_cast<float4*>(wpart + 32 + g * L::PROW + dcol) =
+          make_float4(o[2 * q][0], o[2 * q + 1][0], o[2 * q][1], o[2 * q + 1][1]);
+      *reinterpret_cast<float4*>(wpart + 32 + (g + 8) * L::PROW + dcol) =
+          make_float4(o[2 * q][2], o[2 * q + 1][2], o[2 * q][3], o[2 * q + 1][3]);
     }
   }
   // per-head merge factors of the pairs, once: fac[w][h] = 2^(m_w - M_h)
@@ -507,13 +510,13 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   if (threadIdx.x < 16) {
     const int h = threadIdx.x;
     float M = -INFINITY;
-    for (int w = 0; w < L::NP; ++w) M = fmaxf(M, cmb[w * (L::PART / 4) + h]);
+    for (int w = 0; w < L::NP; ++w) M = fmaxf(M, cmb[w * (L::PPART / 4) + h]);
     float Ls = 0.f;
     for (int w = 0; w < L::NP; ++w) {
-      const float mw = cmb[w * (L::PART / 4) + h];
+      const float mw = cmb[w * (L::PPART / 4) + h];
       const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
       fac[w][h] = f;
-      Ls += cmb[w * (L::PART / 4) + 16 + h] * f;
+      Ls += cmb[w * (L::PPART / 4) + 16 + h] * f;
     }
     float* dst = PARTIALS ? p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D) : mine;
     dst[h] = M;
@@ -524,10 +527,11 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
     float* dst = PARTIALS ? p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D) : mine;
     for (int e4 = threadIdx.x; e4 < 16 * D / 4; e4 += blockDim.x) {
       const int h = (e4 * 4) / D;
+      const int src = h * L::PROW + (e4 * 4) % D;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < L::NP; ++w) {
-        const float4 v = reinterpret_cast<const float4*>(cmb + w * (L::PART / 4) + 32)[e4];
+        const float4 v = *reinterpret_cast<const float4*>(cmb + w * (L::PPART / 4) + 32 + src);
         const float f = fac[w][h];
         acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
       }

@@ -6,31 +6,32 @@
 // forced into the selection and 1024 high-scoring out-of-window tokens added;
 // 10100.com article -- *at most* 1024 (fewer candidates: take them all).
 //
-// One CTA (512 threads) per query row.  Scores are >= 0, so their fp32 bit
-// patterns order like the values.  The k-th largest pattern T is found by a
-// range select that adapts to the row: the first pass records min and max,
-// then each histogram pass splits the current range [lo, hi] into at most
-// 4096 equal bins and keeps the bin that holds the k-th element, so rows whose
-// scores are nearly equal (near-uniform attention) still spread over the bins
-// and 2-3 passes finish.  Keys are then marked in a bitmap over positions --
-// ties at T go to the smaller positions -- and written in ascending order by a
-// block-wide popcount scan, so no sort is needed.  Rows of up to 32768
-// candidates live in shared memory after one read; longer rows are read again
-// for one histogram and then only the candidates of the kept bin are
-// collected into shared memory.
+// One CTA of 256 threads per query row, four CTAs per SM, so one row's
+// barriers and waits overlap the other rows' streaming.  Scores are >= 0, so
+// their fp32 bit patterns order like the values.  The k-th largest pattern T
+// is found by a range select: each pass splits the current pattern range
+// [lo, hi] into at most 2048 equal bins, histograms the candidates (rows are
+// re-read from L2 rather than cached in shared memory) and keeps the bin that
+// holds the k-th element, so rows whose scores are nearly equal still spread
+// over the bins.  As soon as every element that can still be chosen fits a
+// 2048-entry list, one more pass collects them and the remaining passes touch
+// only the list.  The selection is then every key above T plus the first keys
+// equal to T in position order (ties go to the smaller position); it is
+// marked in a bitmap over a window of 32768 positions at a time and written
+// in ascending order by a block-wide popcount scan, so no sort is needed and
+// any row length uses the same 4 KB bitmap.
 #pragma once
 #include "common.cuh"
 
 namespace hs2 {
 
-constexpr int TK_THREADS = 512;
+constexpr int TK_THREADS = 256;
 constexpr int TK_NW = TK_THREADS / 32;
-constexpr int TK_BINS = 4096;
-constexpr int TK_CAP = 8192;          // collected candidates of a long row
-constexpr int TK_CACHE = 32768;       // cached row values (u32); also the long-row bitmap (2^20 bits)
-constexpr int TK_SMALL_BM = TK_CACHE / 32;
-constexpr size_t TK_SMEM = (size_t)TK_BINS * 4 + (size_t)TK_CAP * 8 + (size_t)TK_CACHE * 4 +
-                           (size_t)TK_SMALL_BM * 4 + 256;
+constexpr int TK_BINS = 2048;
+constexpr int TK_CAP = 4096;          // listed candidates (also the sample)
+constexpr int TK_WIN = 32768;         // positions per bitmap window
+constexpr int TK_BMW = TK_WIN / 32;   // bitmap words
+constexpr size_t TK_SMEM = (size_t)TK_BINS * 4 + (size_t)TK_CAP * 8 + (size_t)TK_BMW * 4;
 
 struct TopkParams {
   const float* sigma;    // row r at sigma + r * ld, candidates [0, n_r)
@@ -42,7 +43,15 @@ struct TopkParams {
   int32_t* idx;          // [rows, window + topk]
 };
 
-// Exclusive prefix sum over the CTA's 512 threads; `total` gets the sum.
+__device__ __forceinline__ uint32_t tk_clean(uint32_t u, const DevCtx& ctx) {
+  if (u > 0x7f800000u) {                 // NaN or a negative score: not a probability sum
+    report(ctx, ST_DEVICE_CHECK);
+    return 0u;
+  }
+  return u;
+}
+
+// Exclusive prefix sum over the CTA; `total` gets the sum.  Two barriers.
 __device__ __forceinline__ uint32_t tk_excl_scan(uint32_t v, uint32_t* scratch, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -53,127 +62,89 @@ __device__ __forceinline__ uint32_t tk_excl_scan(uint32_t v, uint32_t* scratch, 
   }
   if (lane == 31) scratch[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    uint32_t w = lane < TK_NW ? scratch[lane] : 0;
+  uint32_t before = 0, tot = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < TK_NW) scratch[TK_NW + lane] = w;
+  for (int w = 0; w < TK_NW; ++w) {
+    const uint32_t s = scratch[w];
+    before += w < warp ? s : 0u;
+    tot += s;
   }
+  total = tot;
   __syncthreads();
-  total = scratch[2 * TK_NW - 1];
-  const uint32_t r = (warp ? scratch[TK_NW + warp - 1] : 0) + x - v;
-  __syncthreads();
-  return r;
+  return before + x - v;
 }
 
-// In a histogram of nbins (<= 4096) bins, the bin b holding the k-th largest
-// element: above(b) < k <= above(b) + hist[b]; res = {b, above(b), hist[b]}.
-__device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int nbins, uint32_t k,
-                                            uint32_t* scratch, uint32_t* res) {
-  constexpr int PER = TK_BINS / TK_THREADS;
-  const int lo = threadIdx.x * PER;
-  uint32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) local += (lo + i < nbins) ? hist[lo + i] : 0u;
+// Block-wide sum (one barrier pair).
+__device__ __forceinline__ uint32_t tk_sum(uint32_t v, uint32_t* scratch) {
   uint32_t total;
-  const uint32_t excl = tk_excl_scan(local, scratch, total);
-  uint32_t above = total - excl - local;        // elements in bins above this range
-  if (local > 0 && above < k && k <= above + local) {
-    for (int b = lo + PER - 1; b >= lo; --b) {
-      const uint32_t h = (b < nbins) ? hist[b] : 0u;
-      if (above + h >= k) {
-        res[0] = (uint32_t)b;
-        res[1] = above;
-        res[2] = h;
-        break;
-      }
-      above += h;
-    }
-  }
-  __syncthreads();
-}
-
-// Ordered positions of set bits: out[j] = position of the j-th set bit (j < limit).
-__device__ __forceinline__ uint32_t tk_emit_bitmap(const uint32_t* bm, int64_t n, int32_t* out,
-                                                   uint32_t limit, uint32_t* scratch) {
-  const int64_t words = (n + 31) >> 5;
-  const int64_t wpt = (words + TK_THREADS - 1) / TK_THREADS;
-  const int64_t w0 = threadIdx.x * wpt;
-  const int64_t w1 = min(words, w0 + wpt);
-  uint32_t local = 0;
-  for (int64_t w = w0; w < w1; ++w) local += __popc(bm[w]);
-  uint32_t total;
-  uint32_t pos = tk_excl_scan(local, scratch, total);
-  for (int64_t w = w0; w < w1; ++w) {
-    uint32_t bits = bm[w];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (pos < limit) out[pos] = (int32_t)(w * 32 + b);
-      ++pos;
-    }
-  }
+  tk_excl_scan(v, scratch, total);
   return total;
 }
 
-// Position of the r-th (1-based) set bit of the bitmap (INT64_MAX if none).
-__device__ __forceinline__ int64_t tk_nth_bit(const uint32_t* bm, int64_t n, uint32_t r,
-                                              uint32_t* scratch, int64_t* res) {
-  const int64_t words = (n + 31) >> 5;
-  const int64_t wpt = (words + TK_THREADS - 1) / TK_THREADS;
-  const int64_t w0 = threadIdx.x * wpt;
-  const int64_t w1 = min(words, w0 + wpt);
-  uint32_t local = 0;
-  for (int64_t w = w0; w < w1; ++w) local += __popc(bm[w]);
-  uint32_t total;
-  uint32_t before = tk_excl_scan(local, scratch, total);
-  if (local > 0 && before < r && r <= before + local) {
-    for (int64_t w = w0; w < w1; ++w) {
-      uint32_t bits = bm[w];
-      const uint32_t c = __popc(bits);
-      if (before + c >= r) {
-        for (uint32_t j = before;; ++j) {
-          const int b = __ffs(bits) - 1;
-          bits &= bits - 1;
-          if (j + 1 == r) { *res = w * 32 + b; break; }
+// In a histogram of nb (<= TK_BINS) bins, the bin b holding the k-th largest
+// element: above(b) < k <= above(b) + hist[b]; res = {b, above(b), hist[b]}.
+// Warp w owns bins [256w, 256w + 256) and reads them lane-interleaved.
+__device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int nb, uint32_t k, uint32_t* scratch,
+                                            uint32_t* res) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int PER = TK_BINS / TK_NW / 32;          // 8 rows of 32 bins per warp
+  const int base = warp * (TK_BINS / TK_NW);
+  uint32_t v[PER];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int bin = base + 32 * j + lane;
+    v[j] = bin < nb ? hist[bin] : 0u;
+    mine += v[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if (lane == 0) scratch[warp] = mine;
+  __syncthreads();
+  uint32_t above = 0;
+#pragma unroll
+  for (int w = 0; w < TK_NW; ++w) above += w > warp ? scratch[w] : 0u;
+  if (above < k && k <= above + mine) {
+#pragma unroll
+    for (int j = PER - 1; j >= 0; --j) {
+      uint32_t x = v[j];                               // inclusive suffix over lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+      }
+      const uint32_t rowsum = __shfl_sync(0xffffffffu, x, 0);
+      if (above + rowsum >= k) {
+        if (above + x - v[j] < k && k <= above + x) {
+          res[0] = (uint32_t)(base + 32 * j + lane);
+          res[1] = above + x - v[j];
+          res[2] = v[j];
         }
         break;
       }
-      before += c;
+      above += rowsum;
     }
   }
   __syncthreads();
-  return *res;
 }
 
-__device__ __forceinline__ uint32_t tk_clean(uint32_t u, const DevCtx& ctx) {
-  if (u > 0x7f800000u) {                 // NaN or a negative score: not a probability sum
-    report(ctx, ST_DEVICE_CHECK);
-    return 0u;
-  }
-  return u;
-}
-
-// f(i, u) for every i < n: 16-byte streaming loads, 4 in flight per thread
-// (the rows are read once, so they are marked evict-first).
+// f(i, u) for every i in [i0, i1) (i0 a multiple of 4): 16-byte loads, 4 in
+// flight per thread.
 template <typename F>
-__device__ __forceinline__ void tk_stream(const uint32_t* src, int64_t n, F&& f) {
+__device__ __forceinline__ void tk_stream(const uint32_t* src, int64_t i0, int64_t i1, F&& f) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
-  const int64_t n4 = n >> 2;
-  for (int64_t j0 = threadIdx.x; j0 < n4; j0 += 4 * TK_THREADS) {
+  const int64_t j0 = i0 >> 2, j1 = i1 >> 2;
+  for (int64_t jb = j0 + threadIdx.x; jb < j1; jb += 4 * TK_THREADS) {
     uint4 v[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int64_t j = j0 + (int64_t)r * TK_THREADS;
-      if (j < n4) v[r] = __ldcs(s4 + j);
+      const int64_t j = jb + (int64_t)r * TK_THREADS;
+      if (j < j1) v[r] = s4[j];
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int64_t j = j0 + (int64_t)r * TK_THREADS;
-      if (j < n4) {
+      const int64_t j = jb + (int64_t)r * TK_THREADS;
+      if (j < j1) {
         f(4 * j, v[r].x);
         f(4 * j + 1, v[r].y);
         f(4 * j + 2, v[r].z);
@@ -181,20 +152,62 @@ __device__ __forceinline__ void tk_stream(const uint32_t* src, int64_t n, F&& f)
       }
     }
   }
-  for (int64_t i = (n4 << 2) + threadIdx.x; i < n; i += TK_THREADS) f(i, __ldcs(src + i));
+  for (int64_t i = (j1 << 2) + threadIdx.x; i < i1; i += TK_THREADS) f(i, src[i]);
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 1)
+// f(i, u, valid) for every i < n with all lanes converged (lanes past the
+// end pass valid = false): 16-byte loads, 8 in flight per thread.
+template <typename F>
+__device__ __forceinline__ void tk_stream_conv(const uint32_t* src, int64_t n, F&& f, const DevCtx& ctx) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  const int64_t n4 = n >> 2;
+  constexpr int R = 8;
+  for (int64_t jb = 0; jb < n4; jb += R * TK_THREADS) {
+    uint4 v[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t j = jb + threadIdx.x + (int64_t)r * TK_THREADS;
+      v[r] = j < n4 ? s4[j] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t j = jb + threadIdx.x + (int64_t)r * TK_THREADS;
+      const bool ok = j < n4;
+      const uint32_t e[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f(4 * j + q, ok ? tk_clean(e[q], ctx) : 0u, ok);
+    }
+  }
+  for (int64_t i0 = n4 << 2; i0 < n; i0 += TK_THREADS) {
+    const int64_t i = i0 + threadIdx.x;
+    const bool ok = i < n;
+    f(i, ok ? tk_clean(src[i], ctx) : 0u, ok);
+  }
+}
+
+// Shared-memory histogram add; a warp whose active lanes all hit one bin
+// (concentrated scores) adds once.
+__device__ __forceinline__ void tk_hist_add(uint32_t* hist, bool in, uint32_t bin) {
+  const unsigned act = __ballot_sync(0xffffffffu, in);
+  if (act == 0) return;
+  const int leader = __ffs(act) - 1;
+  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+  if (__all_sync(0xffffffffu, !in || bin == b0)) {
+    if ((threadIdx.x & 31) == leader) atomicAdd(&hist[b0], (uint32_t)__popc(act));
+  } else if (in) {
+    atomicAdd(&hist[bin], 1u);
+  }
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 4)
 topk_select_kernel(TopkParams p, DevCtx ctx) {
   extern __shared__ __align__(16) uint8_t smem_tk[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_tk);
   uint32_t* cval = hist + TK_BINS;
   int32_t* cpos = reinterpret_cast<int32_t*>(cval + TK_CAP);
-  uint32_t* cache = reinterpret_cast<uint32_t*>(cpos + TK_CAP);
-  uint32_t* small_bm = cache + TK_CACHE;
-  __shared__ uint32_t scratch[2 * TK_NW];
+  uint32_t* bm = reinterpret_cast<uint32_t*>(cpos + TK_CAP);
+  __shared__ uint32_t scratch[TK_NW];
   __shared__ uint32_t res[3];
-  __shared__ uint32_t red[2 * TK_NW];
   __shared__ uint32_t ncand;
   __shared__ int64_t pstar;
 
@@ -204,7 +217,6 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
   const uint32_t k = (uint32_t)p.topk;
   int32_t* out = p.idx + row * (int64_t)(W + p.topk);
   const int64_t n = max((int64_t)0, pos - W + 1);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   for (int w = threadIdx.x; w < W; w += TK_THREADS) {
     const int64_t v = pos - W + 1 + w;
@@ -215,154 +227,225 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
     return;
   }
   const uint32_t* src = reinterpret_cast<const uint32_t*>(p.sigma + row * p.ld);
-  const bool cached = n <= TK_CACHE;
 
-  // ---- pass A: min and max (and the row into shared memory if it fits)
-  uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
-  tk_stream(src, n, [&](int64_t i, uint32_t raw) {
-    const uint32_t u = tk_clean(raw, ctx);
-    if (cached) cache[i] = u;
-    lmin = min(lmin, u);
-    lmax = max(lmax, u);
-  });
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
-    lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-  }
-  if (lane == 0) {
-    red[warp] = lmin;
-    red[TK_NW + warp] = lmax;
-  }
-  __syncthreads();
-  uint32_t lo = red[0], hi = red[TK_NW];
-  for (int w = 1; w < TK_NW; ++w) {
-    lo = min(lo, red[w]);
-    hi = max(hi, red[TK_NW + w]);
-  }
+  // every candidate >= v -> the list (stops writing past TK_CAP; ncand
+  // still counts them all)
+  auto collect = [&](uint32_t v) {
+    if (threadIdx.x == 0) ncand = 0;
+    __syncthreads();
+    tk_stream_conv(src, n, [&](int64_t i, uint32_t u, bool valid) {
+      const bool take = valid && u >= v;
+      const unsigned act = __ballot_sync(0xffffffffu, take);
+      if (act == 0) return;
+      const int lane = threadIdx.x & 31, leader = __ffs(act) - 1;
+      uint32_t base = 0;
+      if (lane == leader) base = atomicAdd(&ncand, (uint32_t)__popc(act));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      const uint32_t slot = base + __popc(act & ((1u << lane) - 1u));
+      if (take && slot < (uint32_t)TK_CAP) {
+        cval[slot] = u;
+        cpos[slot] = (int32_t)i;
+      }
+    }, ctx);
+    __syncthreads();
+  };
 
-  // ---- range select
-  bool listed = false;           // long row whose candidates sit in cval/cpos
-  uint32_t krem = k, in_range = (uint32_t)n;
-  for (int pass = 0; hi > lo; ++pass) {
-    const uint32_t span = hi - lo;
-    const int sh = max(0, 32 - __clz((int)span) - 12);   // (span >> sh) < 4096
-    const int nb = (int)(span >> sh) + 1;
-    for (int b = threadIdx.x; b < nb; b += TK_THREADS) hist[b] = 0;
-    __syncthreads();
-    if (listed) {
-      for (uint32_t c = threadIdx.x; c < ncand; c += TK_THREADS) {
-        const uint32_t u = cval[c];
-        if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
-      }
-    } else if (cached) {
-      for (int64_t i = threadIdx.x; i < n; i += TK_THREADS) {
-        const uint32_t u = cache[i];
-        if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
-      }
-    } else {
-      tk_stream(src, n, [&](int64_t, uint32_t raw) {
-        const uint32_t u = tk_clean(raw, ctx);
-        if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
-      });
-    }
-    __syncthreads();
-    tk_find_bin(hist, nb, krem, scratch, res);
-    const uint32_t b = res[0], above = res[1];
-    in_range = res[2];
-    const uint32_t nlo = lo + (b << sh);
-    const uint32_t nhi = (sh >= 32 || nlo + ((1u << sh) - 1u) > hi || nlo + ((1u << sh) - 1u) < nlo)
-                             ? hi : nlo + ((1u << sh) - 1u);
-    krem -= above;
-    lo = nlo;
-    hi = nhi;
-    if (!listed && k - krem + in_range <= (uint32_t)TK_CAP) {
-      // keep only the elements >= lo (all that can still be chosen): the next
-      // passes and the marking then touch about k elements, not the row
-      if (threadIdx.x == 0) ncand = 0;
+  // ---- range select: the pattern of the r-th largest candidate.  On
+  // return lo == hi is that pattern, krem how many of the r are equal to it
+  // and in_range how many candidates equal it.  Over the list when `listed`,
+  // else over the row, which is collected into the list as soon as every
+  // element that can still be chosen fits it.
+  bool listed = false;                      // candidates >= lo sit in cval/cpos
+  uint32_t lo, hi, krem, in_range;
+  auto range_select = [&](uint32_t r, uint32_t count) {
+    lo = 0u;
+    hi = 0x7f800000u;
+    krem = r;
+    in_range = count;
+    while (hi > lo) {
+      const uint32_t span = hi - lo;
+      const int sh = max(0, 32 - __clz((int)span) - 11);   // (span >> sh) < 2048
+      const int nb = (int)(span >> sh) + 1;
+      for (int b = threadIdx.x; b < nb; b += TK_THREADS) hist[b] = 0;
       __syncthreads();
-      const uint32_t clo = lo;
-      auto take = [&](int64_t i, uint32_t u) {
-        if (u >= clo) {               // at most TK_CAP of them (counted above)
-          const uint32_t slot = atomicAdd(&ncand, 1u);
-          cval[slot] = u;
-          cpos[slot] = (int32_t)i;
+      if (listed) {
+        const uint32_t m = ncand;
+        for (uint32_t c0 = 0; c0 < m; c0 += TK_THREADS) {
+          const uint32_t c = c0 + threadIdx.x;
+          const uint32_t u = c < m ? cval[c] : 0u;
+          const bool in = c < m && u >= lo && u <= hi;
+          tk_hist_add(hist, in, (u - lo) >> sh);
         }
-      };
-      if (cached) {
-        for (int64_t i = threadIdx.x; i < n; i += TK_THREADS) take(i, cache[i]);
       } else {
-        tk_stream(src, n, [&](int64_t i, uint32_t raw) { take(i, tk_clean(raw, ctx)); });
+        tk_stream_conv(src, n, [&](int64_t, uint32_t u, bool valid) {
+          const bool in = valid && u >= lo && u <= hi;
+          tk_hist_add(hist, in, (u - lo) >> sh);
+        }, ctx);
       }
       __syncthreads();
-      listed = true;
+      tk_find_bin(hist, nb, krem, scratch, res);
+      const uint32_t b = res[0], above = res[1];
+      in_range = res[2];
+      const uint32_t nlo = lo + (b << sh);
+      const uint32_t top = nlo + ((1u << sh) - 1u);
+      lo = nlo;
+      hi = (top > hi || top < nlo) ? hi : top;
+      krem -= above;
+      if (!listed && r - krem + in_range <= (uint32_t)TK_CAP) {
+        collect(lo);                         // exactly r - krem + in_range of them
+        listed = true;
+      }
+    }
+  };
+
+  // ---- a bound from a sample: blocks of 128 candidates, every sb-th block,
+  // at most TK_CAP of them.  Its pattern V at rank k*m/n + delta (delta a
+  // few standard deviations of that rank) lies below the row's k-th largest
+  // for any row without extreme structure; one pass then lists every
+  // candidate >= V.  Rows where that fails (fewer than k listed, or more
+  // than the list holds) fall back to the range select over the row.
+  {
+    const int64_t nblk = (n + 127) / 128;
+    const int64_t sb = (nblk + (TK_CAP / 128) - 1) / (TK_CAP / 128);
+    const int64_t nsb = (nblk + sb - 1) / sb;           // sampled blocks
+    const uint32_t m = (uint32_t)(nsb * 128 < (int64_t)TK_CAP ? nsb * 128 : (int64_t)TK_CAP);
+    {
+      constexpr int R = TK_CAP / (4 * TK_THREADS);      // 16-byte loads per thread, all in flight
+      uint4 v[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t q = 4 * (threadIdx.x + r * TK_THREADS);
+        const int64_t i = (int64_t)(q / 128) * sb * 128 + (q % 128);
+        v[r] = make_uint4(0u, 0u, 0u, 0u);               // padding of a short last block ranks last
+        if (q < m) {
+          if (i + 3 < n) {
+            v[r] = reinterpret_cast<const uint4*>(src)[i >> 2];
+          } else {
+            if (i < n) v[r].x = src[i];
+            if (i + 1 < n) v[r].y = src[i + 1];
+            if (i + 2 < n) v[r].z = src[i + 2];
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t q = 4 * (threadIdx.x + r * TK_THREADS);
+        if (q < m) {
+          const int64_t i = (int64_t)(q / 128) * sb * 128 + (q % 128);
+          *reinterpret_cast<uint4*>(cval + q) = make_uint4(tk_clean(v[r].x, ctx), tk_clean(v[r].y, ctx),
+                                                           tk_clean(v[r].z, ctx), tk_clean(v[r].w, ctx));
+          *reinterpret_cast<int4*>(cpos + q) = make_int4((int)i, (int)i + 1, (int)i + 2, (int)i + 3);
+        }
+      }
+    }
+    if (threadIdx.x == 0) ncand = sb == 1 ? (uint32_t)n : m;
+    __syncthreads();
+    listed = true;
+    if (sb == 1) {
+      range_select(k, (uint32_t)n);                    // the whole row is the sample
+    } else {
+      const float ks = (float)k * (float)m / (float)n;
+      const uint32_t rv = min(m, (uint32_t)(ks + 4.f * sqrtf(ks) + 8.f));
+      range_select(rv, m);
+      const uint32_t V = lo;
+      collect(V);
+      if (ncand >= k && ncand <= (uint32_t)TK_CAP) {
+        range_select(k, ncand);
+      } else {
+        listed = false;
+        range_select(k, (uint32_t)n);
+      }
     }
   }
-  const uint32_t T = lo;          // the k-th largest score pattern
-  const uint32_t need_eq = krem;  // how many keys equal to T are taken
+  const uint32_t T = lo;            // the k-th largest score pattern
+  const uint32_t need_eq = krem;    // how many keys equal to T are taken
   const uint32_t eq_count = in_range;
 
-  // ---- mark and emit in position order (a listed row no longer needs the cache)
-  uint32_t* bm = (cached && !listed) ? small_bm : cache;
-  const int64_t words = (n + 31) >> 5;
-  if (threadIdx.x == 0) pstar = INT64_MAX;
-  if (listed) {
-    for (int64_t w = threadIdx.x; w < words; w += TK_THREADS) bm[w] = 0;
-    __syncthreads();
-    if (need_eq < eq_count) {
-      for (uint32_t c = threadIdx.x; c < ncand; c += TK_THREADS)
-        if (cval[c] == T) atomicOr(&bm[cpos[c] >> 5], 1u << (cpos[c] & 31));
-      __syncthreads();
-      tk_nth_bit(bm, n, need_eq, scratch, &pstar);
-      for (int64_t w = threadIdx.x; w < words; w += TK_THREADS) bm[w] = 0;
-      __syncthreads();
+  // g(i, u) over the candidates at positions [w0, w1)
+  auto each = [&](int64_t w0, int64_t w1, auto&& g) {
+    if (listed) {
+      const uint32_t m = ncand;
+      for (uint32_t c = threadIdx.x; c < m; c += TK_THREADS) {
+        const int64_t i = cpos[c];
+        if (i >= w0 && i < w1) g(i, cval[c]);
+      }
+    } else {
+      tk_stream(src, w0, w1, [&](int64_t i, uint32_t raw) { g(i, tk_clean(raw, ctx)); });
     }
-    const int64_t pcut = pstar;
-    for (uint32_t c = threadIdx.x; c < ncand; c += TK_THREADS) {
-      const uint32_t u = cval[c];
-      if (u > T || (u == T && cpos[c] <= pcut)) atomicOr(&bm[cpos[c] >> 5], 1u << (cpos[c] & 31));
-    }
-  } else if (!cached) {
-    // long row that never fit the candidate list: mark straight from global
-    for (int64_t w = threadIdx.x; w < words; w += TK_THREADS) bm[w] = 0;
+  };
+  auto clear_bm = [&]() {
+    for (int w = threadIdx.x; w < TK_BMW; w += TK_THREADS) bm[w] = 0u;
     __syncthreads();
-    if (need_eq < eq_count) {
-      tk_stream(src, n, [&](int64_t i, uint32_t raw) {
-        if (tk_clean(raw, ctx) == T) atomicOr(&bm[i >> 5], 1u << (i & 31));
+  };
+
+  // ---- the tie cut: position of the need_eq-th key equal to T
+  int64_t pcut = INT64_MAX;
+  if (need_eq < eq_count) {
+    uint32_t seen = 0;
+    for (int64_t w0 = 0; w0 < n; w0 += TK_WIN) {
+      const int64_t w1 = min(n, w0 + TK_WIN);
+      clear_bm();
+      each(w0, w1, [&](int64_t i, uint32_t u) {
+        if (u == T) atomicOr(&bm[(i - w0) >> 5], 1u << ((i - w0) & 31));
       });
       __syncthreads();
-      tk_nth_bit(bm, n, need_eq, scratch, &pstar);
-      for (int64_t w = threadIdx.x; w < words; w += TK_THREADS) bm[w] = 0;
-      __syncthreads();
-    }
-    const int64_t pcut = pstar;
-    tk_stream(src, n, [&](int64_t i, uint32_t raw) {
-      const uint32_t u = tk_clean(raw, ctx);
-      if (u > T || (u == T && i <= pcut)) atomicOr(&bm[i >> 5], 1u << (i & 31));
-    });
-  } else {
-    // cached row: a warp covers 32 consecutive positions = one bitmap word
-    __syncthreads();
-    if (need_eq < eq_count) {
-      for (int64_t i0 = 0; i0 < n; i0 += TK_THREADS) {
-        const int64_t i = i0 + threadIdx.x;
-        const unsigned w = __ballot_sync(0xffffffffu, i < n && cache[i] == T);
-        if (lane == 0 && i < n) bm[i >> 5] = w;
+      const uint4 wv = reinterpret_cast<const uint4*>(bm)[threadIdx.x];
+      const uint32_t cnt = __popc(wv.x) + __popc(wv.y) + __popc(wv.z) + __popc(wv.w);
+      uint32_t tot;
+      const uint32_t before = tk_excl_scan(cnt, scratch, tot);
+      const uint32_t r = need_eq - seen;     // rank wanted within this window (1-based)
+      if (r <= tot) {
+        if (before < r && r <= before + cnt) {
+          uint32_t left = r - before;
+          const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t c = __popc(ws[q]);
+            if (left > 0 && left <= c) {
+              uint32_t bits = ws[q];
+              for (uint32_t j = 1; j < left; ++j) bits &= bits - 1;
+              pstar = w0 + (int64_t)(threadIdx.x * 4 + q) * 32 + (__ffs(bits) - 1);
+              left = 0;
+            } else if (left > 0) {
+              left -= c;
+            }
+          }
+        }
+        __syncthreads();
+        pcut = pstar;
+        break;
       }
-      __syncthreads();
-      tk_nth_bit(bm, n, need_eq, scratch, &pstar);
-    }
-    const int64_t pcut = pstar;
-    for (int64_t i0 = 0; i0 < n; i0 += TK_THREADS) {
-      const int64_t i = i0 + threadIdx.x;
-      const uint32_t u = i < n ? cache[i] : 0u;
-      const unsigned w = __ballot_sync(0xffffffffu, i < n && (u > T || (u == T && i <= pcut)));
-      if (lane == 0 && i < n) bm[i >> 5] = w;
+      seen += tot;
     }
   }
-  __syncthreads();
-  const uint32_t got = tk_emit_bitmap(bm, n, out + W, k, scratch);
-  if (got != k && threadIdx.x == 0) report(ctx, ST_DEVICE_CHECK);
+
+  // ---- mark and emit in position order, one window at a time
+  uint32_t written = 0;
+  for (int64_t w0 = 0; w0 < n; w0 += TK_WIN) {
+    const int64_t w1 = min(n, w0 + TK_WIN);
+    clear_bm();
+    each(w0, w1, [&](int64_t i, uint32_t u) {
+      if (u > T || (u == T && i <= pcut)) atomicOr(&bm[(i - w0) >> 5], 1u << ((i - w0) & 31));
+    });
+    __syncthreads();
+    const uint4 wv = reinterpret_cast<const uint4*>(bm)[threadIdx.x];
+    const uint32_t cnt = __popc(wv.x) + __popc(wv.y) + __popc(wv.z) + __popc(wv.w);
+    uint32_t tot;
+    uint32_t at = written + tk_excl_scan(cnt, scratch, tot);
+    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t bits = ws[q];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (at < k) out[W + at] = (int32_t)(w0 + (int64_t)(threadIdx.x * 4 + q) * 32 + bit);
+        ++at;
+      }
+    }
+    written += tot;
+  }
+  if (written != k && threadIdx.x == 0) report(ctx, ST_DEVICE_CHECK);
 }
 
 }  // namespace hs2
