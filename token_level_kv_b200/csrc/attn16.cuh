@@ -78,10 +78,11 @@ __device__ __forceinline__ uint32_t swz_off(int row, int unit) {
 // meet in shared memory (double-buffered, one pair barrier per chunk) and both
 // warps add them in the same order, so both hold the same S and run the same
 // online softmax, and each adds P V for its half of d.  Halving O (64 fp32
-// registers a thread) puts 8 warps on an SM where one warp per row fitted 4,
-// which is what hides the gather and mma latencies.  K and V half rows of a
-// chunk travel as separate stages of a per-warp 5-stage cp.async ring
-// (K_c, V_c, K_c+1, ...), up to 4 stages in flight; rows are stored at a
+// registers a thread) puts 8 warps on an SM where one warp per row fitted 4.
+// Q stays in registers as mma A fragments, so shared memory holds only the
+// gather: K and V half rows of a chunk travel as separate stages of a
+// per-warp 6-stage cp.async ring (K_c, V_c, K_c+1, ...), up to 5 stages in
+// flight (the bytes in flight per SM set the gather rate); rows are stored at a
 // D + 16 byte stride, which keeps the ldmatrix loads of 8 rows on 8 different
 // bank groups.  The reference max of the online softmax moves only when a
 // row's max grows by more than 2^8 (lazy rescale of O).
@@ -89,13 +90,12 @@ template <int D>
 struct SpfLayout {
   static constexpr int CH = 16;
   static constexpr int HD = D / 2;                 // dims per warp
-  static constexpr int NST = 5;                    // stages per warp (K or V half rows of one chunk)
+  static constexpr int NST = 6;                    // stages per warp (K or V half rows of one chunk)
   static constexpr int NPAIR = 4;                  // query rows in flight per CTA
   static constexpr int NT = NPAIR * 64;
   static constexpr int ROW = 2 * HD + 16;          // half row + pad
   static constexpr int STAGE = CH * ROW + CH * 4;  // rows + positions
-  static constexpr int Q_BYTES = 16 * HD * 2;      // swizzled half of Q, per warp
-  static constexpr int WARP = NST * STAGE + Q_BYTES;
+  static constexpr int WARP = NST * STAGE;
   static constexpr int XCH = 2 * 2 * 32 * 8 * 4;   // per pair: [chunk parity][half][8 floats x 32 lanes]
   static constexpr size_t SMEM = 2 * NPAIR * (size_t)WARP + NPAIR * (size_t)XCH;
 };
@@ -110,14 +110,10 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
   const int pair = warp >> 1, h = warp & 1;
   const int g = lane >> 2, t = lane & 3;
   uint8_t* wb = smem_spf + warp * L::WARP;
-  uint8_t* sQ = wb + L::NST * L::STAGE;
-  const uint32_t qa = smem_u32(sQ);
   float4* xch = reinterpret_cast<float4*>(smem_spf + 2 * L::NPAIR * L::WARP + pair * L::XCH);
   const int cpi = (p.n_idx + L::CH - 1) / L::CH;
   const int64_t n_rows = p.n_rows;
   const int dcol0 = h * HD;                          // this warp's first dim
-  // Q half row r, 16-byte unit u stored at unit u ^ (r & 7)
-  auto qoff = [](int r, int u) -> uint32_t { return (uint32_t)(r * HD * 2 + ((u ^ (r & 7)) << 4)); };
   auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory"); };
   int xc = 0;                                        // chunks so far (exchange buffer parity)
 
@@ -151,6 +147,7 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
     const int nstages = 2 * cpi;
     {
       const int32_t p0 = ldpos(0), p1 = ldpos(1);
+      const int32_t p2 = ldpos(2);
       issue(0, p0);
       cp_async_commit();
       issue(1, p0);
@@ -159,16 +156,24 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       cp_async_commit();
       if (nstages > 3) issue(3, p1);
       cp_async_commit();
+      if (nstages > 4) issue(4, p2);
+      cp_async_commit();
     }
+    // positions of chunks c + 2 and c + 3 (their stages are issued in chunk c)
     int32_t q1 = ldpos(2), q2 = ldpos(3);
-    // this warp's half of Q (rows >= H are zero)
+    // this warp's half of Q as mma A fragments (rows >= H are zero): per
+    // 16-dim step kk, {Q[g][2t,2t+1], Q[g+8][2t,2t+1], Q[g][2t+8,2t+9], Q[g+8][2t+8,2t+9]}
+    uint32_t qf[HD / 16][4];
     {
-      const __nv_bfloat16* q = p.Q + row * p.H * D + dcol0;
-      for (int u = lane; u < 16 * HD / 8; u += 32) {
-        const int r = u / (HD / 8), un = u % (HD / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < p.H) v = *reinterpret_cast<const uint4*>(q + r * D + un * 8);
-        *reinterpret_cast<uint4*>(sQ + qoff(r, un)) = v;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(p.Q + (row * p.H + g) * D + dcol0) + t;
+      const uint32_t* q1 = q0 + 8 * (D / 2);
+      const bool h0 = g < p.H, h1 = g + 8 < p.H;
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        qf[kk][0] = h0 ? q0[kk * 8] : 0u;
+        qf[kk][1] = h1 ? q1[kk * 8] : 0u;
+        qf[kk][2] = h0 ? q0[kk * 8 + 4] : 0u;
+        qf[kk][3] = h1 ? q1[kk * 8 + 4] : 0u;
       }
     }
     float o[HD / 8][4];
@@ -177,9 +182,10 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
     for (int c = 0; c < cpi; ++c, ++xc) {
-      // K stage of chunk c: 2c; keep NST-1 stages issued ahead
+      // K stage of chunk c: 2c; keep NST-1 = 5 stages issued ahead
+      static_assert(L::NST == 6, "stage schedule below assumes a 6-stage ring");
       {
-        const int nxt = 2 * c + L::NST - 1;           // K stage of chunk c + 2
+        const int nxt = 2 * c + L::NST - 1;           // V stage of chunk c + 2
         if (nxt < nstages) issue(nxt, q1);
         cp_async_commit();
       }
@@ -192,17 +198,13 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
       float s4[4][4] = {};
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
-        uint32_t a[4], b[4];
-        {
-          const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(a, qa + qoff(r, kk * 2 + (lane >> 4)));
-        }
+        uint32_t b[4];
         {
           const int key = (lane & 7) + (lane >> 4) * 8;
           ldsm_x4(b, ka + key * L::ROW + (kk * 2 + ((lane >> 3) & 1)) * 16);
         }
-        mma_bf16_16816(s4[(kk & 1) * 2 + 0], a, b[0], b[1]);
-        mma_bf16_16816(s4[(kk & 1) * 2 + 1], a, b[2], b[3]);
+        mma_bf16_16816(s4[(kk & 1) * 2 + 0], qf[kk], b[0], b[1]);
+        mma_bf16_16816(s4[(kk & 1) * 2 + 1], qf[kk], b[2], b[3]);
       }
       // exchange the partials; S = S_half0 + S_half1 in both warps
       float s[2][4];
@@ -237,8 +239,8 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
         }
       __syncwarp();            // K stage fully read: it is reissued below
       {
-        const int nxt = 2 * c + L::NST;               // V stage of chunk c + 2
-        if (nxt < nstages) issue(nxt, q1);
+        const int nxt = 2 * c + L::NST;               // K stage of chunk c + 3
+        if (nxt < nstages) issue(nxt, q2);
         cp_async_commit();
       }
       q1 = q2;

@@ -14,14 +14,15 @@
 // TMEM lane is one key and its columns hold every head of every query: the sum
 // over heads is thread-local (no shuffles).  K streams through a ring of
 // 64-column TMA boxes (16 KB); the 256-row Q block stays resident.  TMEM: two
-// S^T buffers of 256 columns.  Eight epilogue warps (two per TMEM lane
-// quarter, each taking half of the queries) write sigma rows coalesced.
+// S^T buffers of 256 columns.  Sixteen epilogue warps (four per TMEM lane
+// quarter, each taking a quarter of the queries) write sigma rows coalesced;
+// with fewer the epilogue, not the tensor pipe, set the pace.
 #pragma once
 #include "common.cuh"
 
 namespace hs2 {
 
-constexpr int SG_THREADS = 320;
+constexpr int SG_THREADS = 576;     // TMA warp, MMA warp, 16 epilogue warps
 constexpr int SG_STAGES = 5;
 
 template <int D>
@@ -82,7 +83,7 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 256);
+      mbar_init(&s_free[i], SG_THREADS - 64);
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -172,8 +173,8 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
     }
   } else {
     const int e = warp - 2;
-    const int quarter = warp & 3;
-    const int half = e >> 2;
+    const int quarter = warp & 3;                  // TMEM lanes a warp may read: 32 * (warp % 4)
+    const int part = e >> 2;                       // columns [64 * part, 64 * part + 64)
     const int kl = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int j = 0; j < n_kt; ++j) {
@@ -182,15 +183,15 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
       tc_fence_after();
       const int64_t key = (int64_t)j * 128 + kl;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 64) {
-        float v[64];
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        float v[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(lane_base + buf * 256 + half * 128 + c0 + c * 16, v + c * 16);
+        for (int c = 0; c < 2; ++c) tmem_ld16(lane_base + buf * 256 + part * 64 + c0 + c * 16, v + c * 16);
         tmem_wait_ld();
-        // column half*128 + c0 + i  <->  (query (half*128 + c0 + i) / H, head i % H)
+        // column part*64 + c0 + i  <->  (query (part*64 + c0 + i) / H, head i % H)
 #pragma unroll
-        for (int qi = 0; qi < 64 / H; ++qi) {
-          const int col = half * 128 + c0 + qi * H;
+        for (int qi = 0; qi < 32 / H; ++qi) {
+          const int col = part * 64 + c0 + qi * H;
           const int64_t tq = g0 + col / H;
           const int64_t pq = p.q_start + tq;
           const float* ml = sML + (size_t)col * 2;

@@ -8,18 +8,24 @@
 //
 // One CTA of 256 threads per query row, four CTAs per SM, so one row's
 // barriers and waits overlap the other rows' streaming.  Scores are >= 0, so
-// their fp32 bit patterns order like the values.  The k-th largest pattern T
-// is found by a range select: each pass splits the current pattern range
-// [lo, hi] into at most 2048 equal bins, histograms the candidates (rows are
-// re-read from L2 rather than cached in shared memory) and keeps the bin that
-// holds the k-th element, so rows whose scores are nearly equal still spread
-// over the bins.  As soon as every element that can still be chosen fits a
-// 2048-entry list, one more pass collects them and the remaining passes touch
-// only the list.  The selection is then every key above T plus the first keys
-// equal to T in position order (ties go to the smaller position); it is
-// marked in a bitmap over a window of 32768 positions at a time and written
-// in ascending order by a block-wide popcount scan, so no sort is needed and
-// any row length uses the same 4 KB bitmap.
+// their fp32 bit patterns order like the values.
+//   1. A sample of the row (every sb-th block of 128 candidates, at most 2048)
+//      is read into shared memory and its pattern V at rank
+//      k*m/n + 4*sqrt(k*m/n) + 8 found: below the row's k-th largest unless the
+//      row is extreme.
+//   2. One pass over the row lists every candidate >= V (one test per 16-byte
+//      group); when that yields between k and 4096 of them, the exact k-th
+//      largest pattern T is found on the list, else (the fallback) on the row.
+//   3. Range select: each pass splits the current pattern range [lo, hi] into
+//      at most 2048 equal bins, histograms the candidates and keeps the bin
+//      that holds the k-th element, so rows whose scores are nearly equal still
+//      spread over the bins.  Over the row (fallback), the survivors are listed
+//      as soon as they fit.
+//   4. The selection is every key above T plus the first keys equal to T in
+//      position order (ties go to the smaller position), marked in a bitmap
+//      over a window of 32768 positions at a time and written in ascending
+//      order by a block-wide popcount scan: no sort, and any row length uses
+//      the same 4 KB bitmap.
 #pragma once
 #include "common.cuh"
 
@@ -28,7 +34,8 @@ namespace hs2 {
 constexpr int TK_THREADS = 256;
 constexpr int TK_NW = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
-constexpr int TK_CAP = 4096;          // listed candidates (also the sample)
+constexpr int TK_CAP = 4096;          // listed candidates
+constexpr int TK_SAMPLE = 2048;       // sampled candidates
 constexpr int TK_WIN = 32768;         // positions per bitmap window
 constexpr int TK_BMW = TK_WIN / 32;   // bitmap words
 constexpr size_t TK_SMEM = (size_t)TK_BINS * 4 + (size_t)TK_CAP * 8 + (size_t)TK_BMW * 4;
@@ -83,46 +90,60 @@ __device__ __forceinline__ uint32_t tk_sum(uint32_t v, uint32_t* scratch) {
 
 // In a histogram of nb (<= TK_BINS) bins, the bin b holding the k-th largest
 // element: above(b) < k <= above(b) + hist[b]; res = {b, above(b), hist[b]}.
-// Warp w owns bins [256w, 256w + 256) and reads them lane-interleaved.
+// Warp w owns bins [256w, 256w + 256) as 8 rows of 32, read lane-interleaved;
+// the 8 row sums are reduced side by side, so only the row holding the bin is
+// scanned.
 __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int nb, uint32_t k, uint32_t* scratch,
                                             uint32_t* res) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int PER = TK_BINS / TK_NW / 32;          // 8 rows of 32 bins per warp
   const int base = warp * (TK_BINS / TK_NW);
-  uint32_t v[PER];
-  uint32_t mine = 0;
+  uint32_t v[PER], rs[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int bin = base + 32 * j + lane;
     v[j] = bin < nb ? hist[bin] : 0u;
-    mine += v[j];
+    rs[j] = v[j];
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int j = 0; j < PER; ++j) rs[j] += __shfl_xor_sync(0xffffffffu, rs[j], o);
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) mine += rs[j];
   if (lane == 0) scratch[warp] = mine;
   __syncthreads();
   uint32_t above = 0;
 #pragma unroll
   for (int w = 0; w < TK_NW; ++w) above += w > warp ? scratch[w] : 0u;
   if (above < k && k <= above + mine) {
+    // the row from the top whose sum reaches k, and its bins
+    uint32_t vj = 0;
+    int jsel = 0;
+    bool found = false;
 #pragma unroll
     for (int j = PER - 1; j >= 0; --j) {
-      uint32_t x = v[j];                               // inclusive suffix over lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
-        if (lane + o < 32) x += y;
-      }
-      const uint32_t rowsum = __shfl_sync(0xffffffffu, x, 0);
-      if (above + rowsum >= k) {
-        if (above + x - v[j] < k && k <= above + x) {
-          res[0] = (uint32_t)(base + 32 * j + lane);
-          res[1] = above + x - v[j];
-          res[2] = v[j];
+      if (!found) {
+        if (above + rs[j] >= k) {
+          found = true;
+          jsel = j;
+          vj = v[j];
+        } else {
+          above += rs[j];
         }
-        break;
       }
-      above += rowsum;
+    }
+    uint32_t x = vj;                                   // inclusive suffix over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+      if (lane + o < 32) x += y;
+    }
+    if (above + x - vj < k && k <= above + x) {
+      res[0] = (uint32_t)(base + 32 * jsel + lane);
+      res[1] = above + x - vj;
+      res[2] = vj;
     }
   }
   __syncthreads();
@@ -185,9 +206,15 @@ __device__ __forceinline__ void tk_stream_conv(const uint32_t* src, int64_t n, F
   }
 }
 
-// Shared-memory histogram add; a warp whose active lanes all hit one bin
-// (concentrated scores) adds once.
+// Shared-memory histogram add.  With AGG (the first pass of a select, where
+// nearly equal scores crowd one bin) a warp whose active lanes all hit one
+// bin adds once; later passes spread over the bins and add directly.
+template <bool AGG>
 __device__ __forceinline__ void tk_hist_add(uint32_t* hist, bool in, uint32_t bin) {
+  if (!AGG) {
+    if (in) atomicAdd(&hist[bin], 1u);
+    return;
+  }
   const unsigned act = __ballot_sync(0xffffffffu, in);
   if (act == 0) return;
   const int leader = __ffs(act) - 1;
@@ -230,23 +257,59 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
 
   // every candidate >= v -> the list (stops writing past TK_CAP; ncand
   // still counts them all)
+  // (one test per 16-byte group: its largest pattern against v)
   auto collect = [&](uint32_t v) {
     if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-    tk_stream_conv(src, n, [&](int64_t i, uint32_t u, bool valid) {
-      const bool take = valid && u >= v;
-      const unsigned act = __ballot_sync(0xffffffffu, take);
-      if (act == 0) return;
-      const int lane = threadIdx.x & 31, leader = __ffs(act) - 1;
-      uint32_t base = 0;
-      if (lane == leader) base = atomicAdd(&ncand, (uint32_t)__popc(act));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      const uint32_t slot = base + __popc(act & ((1u << lane) - 1u));
-      if (take && slot < (uint32_t)TK_CAP) {
-        cval[slot] = u;
-        cpos[slot] = (int32_t)i;
+    auto take4 = [&](int64_t i0, uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3, bool ok) {
+      uint32_t mx = max(max(e0, e1), max(e2, e3));
+      if (ok && mx > 0x7f800000u) {                  // NaN or negative: cleaned (and reported)
+        e0 = tk_clean(e0, ctx); e1 = tk_clean(e1, ctx); e2 = tk_clean(e2, ctx); e3 = tk_clean(e3, ctx);
+        mx = max(max(e0, e1), max(e2, e3));
       }
-    }, ctx);
+      if (ok && mx >= v) {                           // rare: a group with a candidate
+        const uint32_t e[4] = {e0, e1, e2, e3};
+        uint32_t c = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) c += e[q] >= v ? 1u : 0u;
+        uint32_t slot = atomicAdd(&ncand, c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (e[q] >= v) {
+            if (slot < (uint32_t)TK_CAP) {
+              cval[slot] = e[q];
+              cpos[slot] = (int32_t)(i0 + q);
+            }
+            ++slot;
+          }
+      }
+    };
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    const int64_t n4 = n >> 2;
+    constexpr int R = 8;
+    for (int64_t jb = threadIdx.x; jb < n4; jb += R * TK_THREADS) {
+      uint4 w[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t j = jb + (int64_t)r * TK_THREADS;
+        w[r] = j < n4 ? s4[j] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t j = jb + (int64_t)r * TK_THREADS;
+        take4(4 * j, w[r].x, w[r].y, w[r].z, w[r].w, j < n4);
+      }
+    }
+    for (int64_t i = (n4 << 2) + threadIdx.x; i < n; i += TK_THREADS) {
+      const uint32_t u = tk_clean(src[i], ctx);
+      if (u >= v) {
+        const uint32_t slot = atomicAdd(&ncand, 1u);
+        if (slot < (uint32_t)TK_CAP) {
+          cval[slot] = u;
+          cpos[slot] = (int32_t)i;
+        }
+      }
+    }
     __syncthreads();
   };
 
@@ -257,15 +320,19 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
   // element that can still be chosen fits it.
   bool listed = false;                      // candidates >= lo sit in cval/cpos
   uint32_t lo, hi, krem, in_range;
-  auto range_select = [&](uint32_t r, uint32_t count) {
-    lo = 0u;
-    hi = 0x7f800000u;
+  // With win_hi < 0x7f800000 the first pass bins only [win_lo, win_hi] (every
+  // candidate is >= win_lo) plus one overflow bin for the candidates above.
+  auto range_select = [&](uint32_t r, uint32_t count, uint32_t win_lo, uint32_t win_hi) {
+    lo = win_lo;
+    hi = win_hi;
     krem = r;
     in_range = count;
-    while (hi > lo) {
+    bool over = win_hi < 0x7f800000u;                  // first pass only
+    for (int pass = 0; hi > lo || over; ++pass) {
       const uint32_t span = hi - lo;
-      const int sh = max(0, 32 - __clz((int)span) - 11);   // (span >> sh) < 2048
-      const int nb = (int)(span >> sh) + 1;
+      int sh = max(0, 32 - __clz((int)span) - 11);     // (span >> sh) < 2048
+      if (over && (span >> sh) + 2 > (uint32_t)TK_BINS) ++sh;
+      const int nb = (int)(span >> sh) + 1 + (over ? 1 : 0);
       for (int b = threadIdx.x; b < nb; b += TK_THREADS) hist[b] = 0;
       __syncthreads();
       if (listed) {
@@ -273,24 +340,32 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
         for (uint32_t c0 = 0; c0 < m; c0 += TK_THREADS) {
           const uint32_t c = c0 + threadIdx.x;
           const uint32_t u = c < m ? cval[c] : 0u;
-          const bool in = c < m && u >= lo && u <= hi;
-          tk_hist_add(hist, in, (u - lo) >> sh);
+          const bool in = c < m && u >= lo && (u <= hi || over);
+          const uint32_t bin = u > hi ? (uint32_t)(nb - 1) : (u - lo) >> sh;
+          if (pass == 0) tk_hist_add<true>(hist, in, bin);
+          else tk_hist_add<false>(hist, in, bin);
         }
       } else {
         tk_stream_conv(src, n, [&](int64_t, uint32_t u, bool valid) {
           const bool in = valid && u >= lo && u <= hi;
-          tk_hist_add(hist, in, (u - lo) >> sh);
+          tk_hist_add<true>(hist, in, (u - lo) >> sh);
         }, ctx);
       }
       __syncthreads();
       tk_find_bin(hist, nb, krem, scratch, res);
       const uint32_t b = res[0], above = res[1];
       in_range = res[2];
-      const uint32_t nlo = lo + (b << sh);
-      const uint32_t top = nlo + ((1u << sh) - 1u);
-      lo = nlo;
-      hi = (top > hi || top < nlo) ? hi : top;
       krem -= above;
+      if (over && b == (uint32_t)(nb - 1)) {           // the k-th largest lies above the window
+        lo = hi + 1;
+        hi = 0x7f800000u;
+      } else {
+        const uint32_t nlo = lo + (b << sh);
+        const uint32_t top = nlo + ((1u << sh) - 1u);
+        lo = nlo;
+        hi = (top > hi || top < nlo) ? hi : top;
+      }
+      over = false;
       if (!listed && r - krem + in_range <= (uint32_t)TK_CAP) {
         collect(lo);                         // exactly r - krem + in_range of them
         listed = true;
@@ -299,18 +374,18 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
   };
 
   // ---- a bound from a sample: blocks of 128 candidates, every sb-th block,
-  // at most TK_CAP of them.  Its pattern V at rank k*m/n + delta (delta a
+  // at most TK_SAMPLE of them.  Its pattern V at rank k*m/n + delta (delta a
   // few standard deviations of that rank) lies below the row's k-th largest
   // for any row without extreme structure; one pass then lists every
   // candidate >= V.  Rows where that fails (fewer than k listed, or more
   // than the list holds) fall back to the range select over the row.
   {
     const int64_t nblk = (n + 127) / 128;
-    const int64_t sb = (nblk + (TK_CAP / 128) - 1) / (TK_CAP / 128);
+    const int64_t sb = (nblk + (TK_SAMPLE / 128) - 1) / (TK_SAMPLE / 128);
     const int64_t nsb = (nblk + sb - 1) / sb;           // sampled blocks
-    const uint32_t m = (uint32_t)(nsb * 128 < (int64_t)TK_CAP ? nsb * 128 : (int64_t)TK_CAP);
+    const uint32_t m = (uint32_t)(nsb * 128 < (int64_t)TK_SAMPLE ? nsb * 128 : (int64_t)TK_SAMPLE);
     {
-      constexpr int R = TK_CAP / (4 * TK_THREADS);      // 16-byte loads per thread, all in flight
+      constexpr int R = TK_SAMPLE / (4 * TK_THREADS);   // 16-byte loads per thread, all in flight
       uint4 v[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -342,18 +417,23 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
     __syncthreads();
     listed = true;
     if (sb == 1) {
-      range_select(k, (uint32_t)n);                    // the whole row is the sample
+      range_select(k, (uint32_t)n, 0u, 0x7f800000u);   // the whole row is the sample
     } else {
       const float ks = (float)k * (float)m / (float)n;
       const uint32_t rv = min(m, (uint32_t)(ks + 4.f * sqrtf(ks) + 8.f));
-      range_select(rv, m);
+      // the row into L2 while the sample is searched (the next pass reads it all)
+      for (int64_t i = (int64_t)threadIdx.x * 32; i < n; i += 32 * TK_THREADS)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i));
+      range_select(rv, m, 0u, 0x7f800000u);
       const uint32_t V = lo;
       collect(V);
       if (ncand >= k && ncand <= (uint32_t)TK_CAP) {
-        range_select(k, ncand);
+        // T is within a few sample ranks of V: first look 2^16 patterns above it
+        if (V < 0x7f7f0000u) range_select(k, ncand, V, V + 0xffffu);
+        else range_select(k, ncand, 0u, 0x7f800000u);
       } else {
         listed = false;
-        range_select(k, (uint32_t)n);
+        range_select(k, (uint32_t)n, 0u, 0x7f800000u);
       }
     }
   }
