@@ -324,7 +324,8 @@ def run_ours(args, rank, world, dist):
     # algorithmic tensor work per launch; the sparse layer's unique HBM bytes
     # (Q, O, idx, K, V: ~0.7 GB) take less time at the HBM roofline than its
     # FLOPs at the tensor roofline, so its bound is the tensor one
-    work = {"fa_fwd_kernel": full_fl, "select_sigma_kernel": sigma_fl, "sparse_prefill_kernel": sparse_fl1}
+    work = {"fa_fwd_kernel": full_fl, "select_sigma_kernel": sigma_fl, "sparse_prefill_kernel": sparse_fl1,
+            "sparse_tc_kernel": sparse_fl1}
     roof = None
     if dom in work:
         ach = work[dom] / (kern[dom]["avg_ms"] * 1e-3) / 1e12

@@ -148,6 +148,23 @@ def test_sparse_decode_many_sequences(hs2):
     assert max(max_abs(O[b].float().numpy(), ref[b]) for b in range(B)) <= TOL_FP8
 
 
+@pytest.mark.parametrize("n_idx,H,d", [(1920, 16, 256), (2000, 16, 256), (1300, 8, 128), (5, 16, 256)])
+def test_sparse_prefill_index_widths(hs2, n_idx, H, d):
+    """Index rows at the tensor-core kernel's limit (15 tiles of 128 keys), past it (the
+    warp-pair kernel), a ragged H = 8, d = 128 case and a tiny one, each with empty (-1)
+    slots scattered through the row and repeated keys; sampled rows against the oracle."""
+    T = 2200
+    case = synth.make_prefill_case(T, H, d, 128, 64, n_sparse=1, seed=11)
+    rng = np.random.default_rng(n_idx)
+    idx = np.sort(rng.integers(0, T, size=(T, n_idx)), axis=1).astype(np.int32)
+    idx[rng.random((T, n_idx)) < 0.05] = -1
+    idx[:, 0] = np.arange(T)                  # every row keeps one real key
+    O = gpu_sparse_prefill(case.Q_sparse[0], case.K, case.V, idx)
+    rows = list(range(0, T, 173)) + [T - 1]
+    ref = oracle.sparse_attn(case.Q_sparse[0], case.K, case.V, idx, rows)
+    assert max(max_abs(O[t].float().numpy(), ref[t]) for t in rows) <= TOL_BF16
+
+
 # ---------------------------------------------------------------- checks and faults
 
 def test_sparse_prefill_bad_index_is_reported_and_skipped(hs2):

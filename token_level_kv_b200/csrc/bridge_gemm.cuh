@@ -155,7 +155,7 @@ bridge_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      if (!mbar_wait(&tfull[acc], acc_phase, ctx)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, ctx))) break;
       tc_fence_after();
       const int m = tile >> 1;
       const bool is_v = tile & 1;

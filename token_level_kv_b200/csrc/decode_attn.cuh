@@ -203,7 +203,8 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   constexpr int RPI = 32 / UPR;                      // rows per copy instruction (gather)
   auto produce = [&](int i) -> bool {
     const int s = i % L::NS;
-    if (!mbar_wait(&empty[s], (uint32_t)(((i / L::NS) & 1) ^ 1), ctx)) return false;
+    // the warp decides together (a lane that timed out stops all of it)
+    if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], (uint32_t)(((i / L::NS) & 1) ^ 1), ctx))) return false;
     uint8_t* st = ring + s * L::STAGE;
     if (RANGE) {
       const int64_t pos0 = s_begin + (int64_t)i * L::CH;
@@ -315,7 +316,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
       // both warps of the pair reach the pair barrier below on every step and
       // leave the loop together: a timed-out wait still takes part in the
       // exchange (its S is junk) and both warps then see the failure
-      const bool ok = mbar_wait(&full[slot], (uint32_t)((i / L::NS) & 1), ctx);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[slot], (uint32_t)((i / L::NS) & 1), ctx));
       const uint8_t* st = ring + slot * L::STAGE;
       const float* sks = L::kscale(smem, slot);
       const float* svs = sks + L::CH;

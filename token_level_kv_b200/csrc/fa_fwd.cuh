@@ -196,7 +196,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     float x[128];
     for (int j = 0; j < n_kt; ++j) {
       const int s = j & 1;
-      if (!mbar_wait(&s_full[s], (j >> 1) & 1, ctx)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, ctx))) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + s * 128 + c * 32, x + c * 32);
@@ -231,7 +231,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       l = l * alpha + rs;
 
       if (j >= 1) {
-        if (!mbar_wait(p_empty, (j - 1) & 1, ctx)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(p_empty, (j - 1) & 1, ctx))) { ok = false; break; }
         tc_fence_after();
       }
       // P row -> shared memory, K-major 128B swizzle: 2 blocks of 64 keys
@@ -261,7 +261,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(o_final, 0, ctx)) {
+    if (__all_sync(0xffffffffu, ok && mbar_wait(o_final, 0, ctx))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* out = p.O + R * D;

@@ -20,6 +20,7 @@
 #include "fa_fwd.cuh"
 #include "select_sigma.cuh"
 #include "topk.cuh"
+#include "sparse_tc.cuh"
 
 namespace hs2 {
 
@@ -231,10 +232,20 @@ hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O
   return after_launch("attn16_combine_kernel", st);
 }
 
+// Rows of up to 1920 keys run on the tensor cores (sparse_tc_kernel, one CTA
+// per SM); longer ones on the warp-pair kernel (4 rows per SM).
 template <int D>
-hs2_status launch_sparse_prefill(const Attn16Params& p, int grid, cudaStream_t st, const DevCtx& ctx) {
-  hs2_status s = set_smem(sparse_prefill_kernel<D>, SpfLayout<D>::SMEM);
-  if (s != HS2_OK) return s;
+hs2_status launch_sparse_prefill(const Attn16Params& p, int sms, cudaStream_t st, const DevCtx& ctx) {
+  hs2_status s;
+  if ((p.n_idx + 127) / 128 <= StcLayout<D>::MAXT) {
+    if ((s = set_smem(sparse_tc_kernel<D>, StcLayout<D>::SMEM)) != HS2_OK) return s;
+    const int grid = (int)std::min<int64_t>(p.n_rows, sms);
+    prof_begin(st);
+    sparse_tc_kernel<D><<<grid, StcLayout<D>::NT, StcLayout<D>::SMEM, st>>>(p, ctx);
+    return after_launch("sparse_tc_kernel", st);
+  }
+  if ((s = set_smem(sparse_prefill_kernel<D>, SpfLayout<D>::SMEM)) != HS2_OK) return s;
+  const int grid = (int)std::min<int64_t>((p.n_rows + SpfLayout<D>::NPAIR - 1) / SpfLayout<D>::NPAIR, sms);
   prof_begin(st);
   sparse_prefill_kernel<D><<<grid, SpfLayout<D>::NT, SpfLayout<D>::SMEM, st>>>(p, ctx);
   return after_launch("sparse_prefill_kernel", st);
@@ -559,8 +570,7 @@ hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int sms = 0;
   if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
-  const int grid = (int)std::min<int64_t>((Tq + SpfLayout<256>::NPAIR - 1) / SpfLayout<256>::NPAIR, sms);
-  return d == 256 ? launch_sparse_prefill<256>(p, grid, st, ctx) : launch_sparse_prefill<128>(p, grid, st, ctx);
+  return d == 256 ? launch_sparse_prefill<256>(p, sms, st, ctx) : launch_sparse_prefill<128>(p, sms, st, ctx);
 }
 
 hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d, size_t* bytes) {

@@ -179,7 +179,7 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int j = 0; j < n_kt; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(&s_full[buf], (j >> 1) & 1, ctx)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, ctx))) break;
       tc_fence_after();
       const int64_t key = (int64_t)j * 128 + kl;
 #pragma unroll 1
