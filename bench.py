@@ -113,9 +113,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 # DRAM bytes per query row of a launch, from one ncu capture of the kernel as
-# it stands (113.8 MB read + 39.5 MB written by one T = 8192 launch); set to
-# None whenever the kernel changes.
-DRAM_BYTES_PER_ROW = {"sparse_prefill_kernel": (113.825024e6 + 39.492096e6) / 8192}
+# it stands (113.5 MB read + 41.1 MB written by one T = 8192 launch); drop the
+# entry whenever the kernel changes.
+DRAM_BYTES_PER_ROW = {"sparse_tc_kernel": (113.483776e6 + 41.083648e6) / 8192}
 
 
 def prefill_flops(T, H, d, window, topk, n_sparse):

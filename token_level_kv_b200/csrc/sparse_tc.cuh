@@ -15,7 +15,9 @@
 //     [16t, 16t+16) of the row's S buffer; after the softmax it adds
 //     O^T += V_t^T P_t^T (M = 128 dims per half of d -- V read MN-major
 //     straight from the gathered tile --, N = 16 heads, K = 128 keys) into
-//     TMEM columns [480, 480 + 16 * d/128).
+//     TMEM columns [480, 480 + 16 * d/128).  With N = 16 a row takes 288
+//     MMAs, so the issuing thread only adds constants to descriptors built
+//     once per stage.
 //   * Four softmax warps (one TMEM lane quarter each: a thread is one key of
 //     every tile) run an exact two-pass softmax over the whole row: the
 //     per-head maximum over all the row's keys, then p = 2^(s*c - m*c) into
@@ -24,8 +26,11 @@
 //   * Two rows are in flight: the ring carries K(0), K(1), V(0), K(2), V(1), ...
 //     and S^T is double-buffered in TMEM, so row r's softmax overlaps row
 //     r+1's gather and Q K^T products.
+//   * P^T moves tile by tile through a 2-tile ring: the softmax writes tile t
+//     while the tensor cores multiply tile t-1, which leaves shared memory to
+//     a 6-stage gather ring (192 KB in flight).
 // Rows of up to 15 tiles (1920 keys): TMEM 2 x 240 + 32 columns (512 taken),
-// shared memory 4 x 32 KB ring + 60 KB P^T + 2 x 8 KB Q + 2 x 7.5 KB positions.
+// shared memory 6 x 32 KB ring + 2 x 4 KB P^T + 2 x 8 KB Q.
 #pragma once
 #include "attn16.cuh"
 #include "common.cuh"
@@ -37,18 +42,19 @@ struct StcLayout {
   static constexpr int NPROD = 8;                // producer warps (16 key rows of a stage each)
   static constexpr int MMA_WARP = 4 + NPROD;
   static constexpr int NT = (MMA_WARP + 1) * 32; // 4 softmax warps, the producers, 1 MMA warp
-  static constexpr int NSTG = 4;                 // ring stages
+  static constexpr int NSTG = 6;                 // ring stages
   static constexpr int STAGE = 128 * 256;        // 128 keys x 128 dims bf16 (two 16 KB atom columns)
   static constexpr int MAXT = 15;                // tiles of 128 keys per row
   static constexpr int SBUF = 16 * MAXT;         // TMEM columns of one S^T buffer
+  static constexpr int OCOL = 2 * SBUF;          // O^T: 16 columns per half of d
   static constexpr int HALVES = D / 128;         // stages per tile (K or V)
   static constexpr int P_TILE = 16 * 256;        // P^T of one tile: 16 heads x 128 keys bf16
+  static constexpr int NPS = 2;                  // P^T tiles in flight (softmax -> P V products)
   static constexpr int Q_BYTES = 16 * D * 2;     // 16 heads x d, D/64 atom columns of 2 KB
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_P = OFF_RING + NSTG * STAGE;
-  static constexpr int OFF_Q = OFF_P + MAXT * P_TILE;
-  static constexpr int OFF_POS = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_RED = OFF_POS + 2 * MAXT * 128 * 4;
+  static constexpr int OFF_Q = OFF_P + NPS * P_TILE;
+  static constexpr int OFF_RED = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_RED + (2 * 4 * 16 + 2 * 16) * 4;
   static constexpr size_t SMEM = OFF_BAR + 256 + 1024;   // + base alignment
 };
@@ -81,7 +87,6 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
   uint8_t* ring = smem + L::OFF_RING;
   uint8_t* sP = smem + L::OFF_P;
   uint8_t* sQ = smem + L::OFF_Q;
-  int32_t* spos = reinterpret_cast<int32_t*>(smem + L::OFF_POS);      // [2][MAXT][128]
   float* red_m = reinterpret_cast<float*>(smem + L::OFF_RED);        // [4][16]
   float* red_l = red_m + 64;                                          // [4][16]
   float* linv = red_l + 64;                                           // [2][16]
@@ -89,8 +94,9 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
   uint64_t* full = bars;                       // [NSTG] producers' cp.async arrivals
   uint64_t* empty = full + L::NSTG;            // [NSTG] MMA commit
   uint64_t* s_full = empty + L::NSTG;          // [2] S^T of a row complete (per S buffer)
-  uint64_t* p_full = s_full + 2;               // P^T written, S read
-  uint64_t* o_full = p_full + 1;               // O^T of a row complete
+  uint64_t* p_full = s_full + 2;               // [NPS] a P^T tile written (the row's S read)
+  uint64_t* p_empty = p_full + L::NPS;         // [NPS] its products done
+  uint64_t* o_full = p_empty + L::NPS;         // O^T of a row complete
   uint64_t* mma_done = o_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
@@ -107,7 +113,10 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
+    for (int i = 0; i < L::NPS; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_empty[i], 1);
+    }
     mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -163,21 +172,27 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
 #pragma unroll
       for (int i = 0; i < RW / 2; ++i) cp_async16(sa + doff[i], srow[i] + c * 256, (svalid >> i) & 1u);
     };
+    // positions of tile t of a row (lane r < RW: row RW*w + r), loaded one
+    // tile ahead so their latency hides behind the copies; entries outside
+    // [-1, kv_len) are reported (once, in the K pass) and skipped
+    auto ldpos = [&](const int32_t* irow, int t) -> int32_t {
+      const int sl = t * 128 + RW * w + lane;
+      return (t < nT && lane < RW && sl < p.n_idx) ? irow[sl] : -1;
+    };
     // step st: the K stages of row st (st < R), then the V stages of row st-1
     for (int st = 0; st <= R && ok; ++st) {
       if (st < R) {
         const int64_t row = blockIdx.x + (int64_t)st * gridDim.x;
-        int32_t* pos = spos + (st & 1) * (L::MAXT * 128);
         const int32_t* irow = p.idx + row * p.n_idx;
         uint8_t* qb = sQ + (st & 1) * L::Q_BYTES;
+        int32_t nextpos = ldpos(irow, 0);
         for (int t = 0; t < nT && ok; ++t) {
-          const int sl = t * 128 + RW * w + lane;
-          int32_t mypos = (lane < RW && sl < p.n_idx) ? irow[sl] : -1;
+          int32_t mypos = nextpos;
+          nextpos = ldpos(irow, t + 1);
           if (mypos < -1 || mypos >= p.kv_len) {
             report(ctx, ST_DEVICE_CHECK);
             mypos = -1;
           }
-          if (lane < RW) pos[t * 128 + RW * w + lane] = mypos;
           set_rows(reinterpret_cast<const uint8_t*>(p.K), mypos);
           for (int c = 0; c < L::HALVES; ++c) {
             uint8_t* stg = acquire();
@@ -198,9 +213,12 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
         }
       }
       if (st >= 1) {
-        const int32_t* pos = spos + ((st - 1) & 1) * (L::MAXT * 128);
+        const int32_t* irow = p.idx + (blockIdx.x + (int64_t)(st - 1) * gridDim.x) * p.n_idx;
+        int32_t nextpos = ldpos(irow, 0);
         for (int t = 0; t < nT && ok; ++t) {
-          const int32_t mypos = lane < RW ? pos[t * 128 + RW * w + lane] : -1;
+          int32_t mypos = nextpos;
+          nextpos = ldpos(irow, t + 1);
+          if (mypos < -1 || mypos >= p.kv_len) mypos = -1;
           set_rows(reinterpret_cast<const uint8_t*>(p.V), mypos);
           for (int c = 0; c < L::HALVES; ++c) {
             uint8_t* stg = acquire();
@@ -219,22 +237,29 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
       constexpr uint32_t idO = umma_idesc_bf16_amn(128, 16);
       int slot = 0;
       uint32_t phase = 0;
+      int pg = 0;                                     // P^T tiles consumed so far
       bool ok = true, any = false;
+      // descriptors of stage 0 and P^T slot 0, built once (K: K-major; V: MN-major,
+      // 16 KB between 64-dim blocks); the others are a start-address offset away
+      const uint64_t dring0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
+      const uint64_t dvring0 = umma_desc_sw128(smem_u32(ring), 16384, 1024);
+      const uint64_t dpt0 = umma_desc_sw128(smem_u32(sP), 16, 1024);
       for (int st = 0; st <= R && ok; ++st) {
         if (st < R) {
           // S^T_t = K_t Q^T of row st into S buffer st & 1, one stage (128 dims) at a time
-          const uint32_t aQ = smem_u32(sQ + (st & 1) * L::Q_BYTES);
+          // descriptors advance by adding (byte offset >> 4) to the start-address field
+          const uint64_t dQ = umma_desc_sw128(smem_u32(sQ + (st & 1) * L::Q_BYTES), 16, 1024);
           const uint32_t sb = tmem + (st & 1) * L::SBUF;
           for (int t = 0; t < nT && ok; ++t) {
             for (int c = 0; c < L::HALVES; ++c) {
               if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
               fence_proxy_async_smem();              // cp.async (generic) data -> tensor-core reads
               tc_fence_after();
-              const uint32_t aK = smem_u32(ring + slot * L::STAGE);
+              const uint64_t dK = dring0 + (uint64_t)(slot * (L::STAGE >> 4));
 #pragma unroll
               for (int k = 0; k < 8; ++k) {           // 8 steps of 16 dims
-                const uint64_t ad = umma_desc_sw128(aK + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                const uint64_t bd = umma_desc_sw128(aQ + (2 * c + (k >> 2)) * 2048 + (k & 3) * 32, 16, 1024);
+                const uint64_t ad = dK + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4);
+                const uint64_t bd = dQ + (uint64_t)((c * 4096 + (k >> 2) * 2048 + (k & 3) * 32) >> 4);
                 umma_bf16(sb + 16 * t, ad, bd, idS, (c | k) != 0 ? 1u : 0u);
               }
               any = true;
@@ -247,24 +272,26 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
         }
         if (st >= 1) {
           // O^T[half c] += V_t^T P_t^T of row st-1 over each tile's 128 keys
-          if (!mbar_wait(p_full, (st - 1) & 1, ctx)) { ok = false; break; }
-          tc_fence_after();
-          for (int t = 0; t < nT && ok; ++t) {
-            const uint32_t aP = smem_u32(sP + t * L::P_TILE);
+          for (int t = 0; t < nT && ok; ++t, ++pg) {
+            const int ps = pg % L::NPS;
+            if (!mbar_wait(&p_full[ps], (uint32_t)((pg / L::NPS) & 1), ctx)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t dP = dpt0 + (uint64_t)(ps * (L::P_TILE >> 4));
             for (int c = 0; c < L::HALVES; ++c) {
               if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
               fence_proxy_async_smem();
               tc_fence_after();
-              const uint32_t aV = smem_u32(ring + slot * L::STAGE);
+              const uint64_t dV = dvring0 + (uint64_t)(slot * (L::STAGE >> 4));
 #pragma unroll
               for (int k = 0; k < 8; ++k) {           // 8 steps of 16 keys
-                const uint64_t ad = umma_desc_sw128(aV + k * 2048, 16384, 1024);
-                const uint64_t bd = umma_desc_sw128(aP + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024);
-                umma_bf16(tmem + 2 * L::SBUF + 16 * c, ad, bd, idO, (t | k) != 0 ? 1u : 0u);
+                const uint64_t ad = dV + (uint64_t)((k * 2048) >> 4);
+                const uint64_t bd = dP + (uint64_t)(((k >> 2) * 2048 + (k & 3) * 32) >> 4);
+                umma_bf16(tmem + L::OCOL + 16 * c, ad, bd, idO, (t | k) != 0 ? 1u : 0u);
               }
               umma_commit(&empty[slot]);
               if (++slot == L::NSTG) { slot = 0; phase ^= 1; }
             }
+            if (ok) umma_commit(&p_empty[ps]);
           }
           if (!ok) break;
           umma_commit(o_full);
@@ -282,6 +309,7 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
     const float c = p.scale_log2;
     bool ok = true;
+    int pg = 0;                                        // P^T tiles written so far
     // the output of row r (O^T in TMEM -> bf16 O; a thread is one dim)
     auto epilogue = [&](int r) -> bool {
       if (!bar_and(1, 128, mbar_wait(o_full, r & 1, ctx))) return false;
@@ -290,7 +318,7 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
       const float* li = linv + (r & 1) * 16;
       for (int hv = 0; hv < L::HALVES; ++hv) {
         float o[16];
-        tmem_ld16(lane_base + 2 * L::SBUF + 16 * hv, o);
+        tmem_ld16(lane_base + L::OCOL + 16 * hv, o);
         tmem_wait_ld();
         __nv_bfloat16* out = p.O + row * p.H * D + hv * 128 + kl;
 #pragma unroll
@@ -347,18 +375,22 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
         const float mh = fmaxf(fmaxf(red_m[h], red_m[16 + h]), fmaxf(red_m[32 + h], red_m[48 + h]));
         mc[h] = mh == -INFINITY ? 0.f : mh * c;
       }
-      // the previous row's P^T has been read once its O^T is complete
+      // the previous row's O^T must be read before this row's products start
       if (r >= 1 && !epilogue(r - 1)) { ok = false; break; }
-      // pass 2: p = 2^(s*c - m*c), the sums, and P^T (K-major, 128-byte swizzle)
+      // pass 2: p = 2^(s*c - m*c), the sums, and P^T (K-major, 128-byte
+      // swizzle) tile by tile through the P ring
       float l[16];
 #pragma unroll
       for (int h = 0; h < 16; ++h) l[h] = 0.f;
-      for (int t = 0; t < nT; ++t) {
+      for (int t = 0; t < nT; ++t, ++pg) {
+        const int ps = pg % L::NPS;
+        if (!bar_and(1, 128, mbar_wait(&p_empty[ps], (uint32_t)(((pg / L::NPS) & 1) ^ 1), ctx))) { ok = false; break; }
+        tc_fence_after();
         float v[16];
         tmem_ld16(sbuf + 16 * t, v);
         tmem_wait_ld();
         const bool valid = (vmask >> t) & 1u;
-        uint8_t* pt = sP + t * L::P_TILE + (kl >> 6) * 2048;
+        uint8_t* pt = sP + ps * L::P_TILE + (kl >> 6) * 2048;
         const int u8 = (kl & 63) >> 3, e = kl & 7;
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
@@ -366,8 +398,11 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
           l[h] += pv;
           *reinterpret_cast<__nv_bfloat16*>(pt + h * 128 + ((u8 ^ (h & 7)) << 4) + e * 2) = __float2bfloat16_rn(pv);
         }
+        fence_proxy_async_smem();                      // P^T visible to the tensor cores
+        tc_fence_before();
+        mbar_arrive(&p_full[ps]);
       }
-      tc_fence_before();
+      if (!ok) break;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
@@ -384,8 +419,6 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
         const float ls = red_l[h] + red_l[16 + h] + red_l[32 + h] + red_l[48 + h];
         linv[(r & 1) * 16 + h] = ls > 0.f ? 1.f / ls : 0.f;
       }
-      fence_proxy_async_smem();                        // P^T visible to the tensor cores
-      mbar_arrive(p_full);
     }
     if (ok && R > 0) epilogue(R - 1);
   }
