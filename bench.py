@@ -113,9 +113,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 # DRAM bytes per query row of a launch, from one ncu capture of the kernel as
-# it stands (113.5 MB read + 41.1 MB written by one T = 8192 launch); drop the
+# it stands (113.3 MB read + 41.4 MB written by one T = 8192 launch); drop the
 # entry whenever the kernel changes.
-DRAM_BYTES_PER_ROW = {"sparse_tc_kernel": (113.483776e6 + 41.083648e6) / 8192}
+DRAM_BYTES_PER_ROW = {"sparse_tc_kernel": (113.317888e6 + 41.395456e6) / 8192}
 
 
 def prefill_flops(T, H, d, window, topk, n_sparse):
