@@ -12,9 +12,6 @@
 
 namespace hs2 {
 
-constexpr int A16_WARPS = 4;
-constexpr int A16_CH = 16;
-
 struct Attn16Params {
   const __nv_bfloat16* Q;   // [n_rows, H, D]
   const void* K;            // bf16 [kv_len, D]
@@ -64,12 +61,6 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool va
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// bf16 row of D elements, 16-byte unit u stored at unit u ^ (row & 7).
-template <int D>
-__device__ __forceinline__ uint32_t swz_off(int row, int unit) {
-  return (uint32_t)(row * D * 2 + ((unit ^ (row & 7)) << 4));
-}
 
 // Sparse prefill layer (row a6) over the shared bf16 KV.  A PAIR of warps
 // owns one query row; warp half h holds dims [h*D/2, (h+1)*D/2) of Q, of the

@@ -81,13 +81,6 @@ __device__ __forceinline__ uint32_t tk_excl_scan(uint32_t v, uint32_t* scratch, 
   return before + x - v;
 }
 
-// Block-wide sum (one barrier pair).
-__device__ __forceinline__ uint32_t tk_sum(uint32_t v, uint32_t* scratch) {
-  uint32_t total;
-  tk_excl_scan(v, scratch, total);
-  return total;
-}
-
 // In a histogram of nb (<= TK_BINS) bins, the bin b holding the k-th largest
 // element: above(b) < k <= above(b) + hist[b]; res = {b, above(b), hist[b]}.
 // Warp w owns bins [256w, 256w + 256) as 8 rows of 32, read lane-interleaved;
