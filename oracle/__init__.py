@@ -195,8 +195,14 @@ def full_attn_select(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rows: Sequence
 
 def sparse_attn_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx_row: np.ndarray,
                     scale: float) -> np.ndarray:
-    """Sparse layer: softmax attention of its own q over the selected keys only."""
+    """Sparse layer: softmax attention of its own q over the selected keys only.
+
+    An entry that appears twice in the row is attended twice (each slot is one
+    key of the softmax).  A row with no valid entry selects nothing; its output
+    is taken as zero (the empty sum), the library's stated convention."""
     S = idx_row[idx_row >= 0].astype(np.int64)
+    if S.shape[0] == 0:
+        return np.zeros((q.shape[0], V.shape[1]), dtype=np.float64)
     s = (q @ K[S].T) * scale                         # [H, |S|]
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
@@ -242,6 +248,9 @@ def decode_select(Q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ks: np.ndarray,
 def sparse_attn_decode(Qs: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ks: np.ndarray,
                        vs: np.ndarray, idx: np.ndarray, seqs: Sequence[int],
                        scale: Optional[float] = None) -> Dict[int, np.ndarray]:
+    """Sparse layer at decode over the FP8 cache: sequence b's query attends to
+    the rows idx[b] of its OWN cache, key row j being E4M3(Kc[b,j]) * ks[b,j]
+    and value row j being E4M3(Vc[b,j]) * vs[b,j]."""
     d = Qs.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     idx = idx.cpu().numpy() if hasattr(idx, "cpu") else np.asarray(idx)

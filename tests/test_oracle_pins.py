@@ -189,6 +189,37 @@ def test_topk_matches_torch_topk():
         assert r.tau == pytest.approx(float(np.sort(r.sigma[:n_cand])[-k]), rel=0)
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_tau_is_torch_topk_kth_value_with_ties(seed):
+    """tau (the k-th largest candidate score, the centre of the tie margin) is
+    torch.topk's last value, also on rows whose boundary falls inside a run of
+    exactly tied scores (duplicated keys, and K = 0 where every score ties)."""
+    T, H, d, W, k = 60, 3, 8, 4, 7
+    q = _rand((T, H, d), 400 + seed)
+    K = _rand((T, d), 500 + seed)
+    if seed == 3:
+        K[:] = 0.0                                     # every candidate score equal
+    else:
+        for a, b in ((0, 2), (0, 5), (0, 9), (4, 11), (4, 13), (6, 20), (6, 21), (6, 22)):
+            K[b] = K[a]                                # runs of exactly equal scores
+    rows = oracle.full_attn_select(q, K, _rand((T, d), 600 + seed), range(T), 0, W, k)
+    n_ties = 0
+    for t, r in rows.items():
+        n_cand = max(0, t - W + 1)
+        if n_cand <= k:
+            assert r.tau is None
+            continue
+        sc = torch.from_numpy(r.sigma[:n_cand])
+        vals = torch.topk(sc, k).values
+        assert r.tau == float(vals[-1])
+        # the k-th and (k+1)-th values differ unless the boundary sits in a tie run
+        kp1 = float(torch.topk(sc, k + 1).values[-1])
+        n_ties += r.tau == kp1
+        assert r.tau >= kp1
+    if seed == 3:
+        assert n_ties == sum(1 for t in range(T) if t - W + 1 > k)
+
+
 def _brute_force_topk(sigma_c, k):
     """The unique k-subset whose every member outranks every non-member under
     (score, -position) order -- found by trying all subsets."""
@@ -255,6 +286,74 @@ def test_sparse_matches_masked_sdpa():
     ref = _sdpa(qs, K, V, mask=mask)
     for t in range(T):
         assert np.allclose(got[t], ref[t], rtol=1e-12, atol=1e-12)
+
+
+def _fp8_cache(B, N, d, seed, lo, hi):
+    """Random finite E4M3 codes (the two NaN codes avoided) and per-token
+    scales drawn log-uniformly in [lo, hi) -- a different range per call, so a
+    K scale used for V (or the reverse) moves every output."""
+    g = np.random.default_rng(seed)
+    codes = g.integers(0, 0x7E, size=(B, N, d)).astype(np.uint8)
+    codes |= (g.integers(0, 2, size=(B, N, d)) << 7).astype(np.uint8)      # random signs
+    scales = np.exp(g.uniform(np.log(lo), np.log(hi), size=(B, N)))
+    return torch.from_numpy(codes), torch.from_numpy(scales)
+
+
+def _sparse_decode_ref(Qs, Kc, Vc, ks, vs, idx, b, scale):
+    """torch only: dequantise sequence b's cache through torch's own E4M3 type,
+    gather the slots of idx[b] (a repeated slot is gathered twice), fp64 SDPA."""
+    S = torch.from_numpy(idx[b][idx[b] >= 0].astype(np.int64))
+    K = Kc[b].view(torch.float8_e4m3fn).to(torch.float64) * ks[b][:, None]
+    V = Vc[b].view(torch.float8_e4m3fn).to(torch.float64) * vs[b][:, None]
+    q = torch.from_numpy(np.asarray(Qs[b], dtype=np.float64))[:, None, :]          # [H, 1, d]
+    Kg = K.index_select(0, S)[None].expand(q.shape[0], -1, -1)
+    Vg = V.index_select(0, S)[None].expand(q.shape[0], -1, -1)
+    return F.scaled_dot_product_attention(q, Kg, Vg, scale=scale)[:, 0].numpy()
+
+
+def test_sparse_attn_decode_matches_sdpa_over_torch_dequantised_cache():
+    """The sparse decode oracle reads sequence b's own cache rows, K codes with
+    K scales and V codes with V scales: checked against torch's E4M3 decode and
+    fp64 SDPA over the gathered rows, with -1 slots, repeated slots, an empty
+    row and per-sequence scale ranges; then two planted gather mistakes (K and
+    V scales swapped, every sequence reading its neighbour's cache) must fail."""
+    B, N, H, d, n_idx = 4, 90, 4, 16, 24
+    Kc, ks = _fp8_cache(B, N, d, 40, 1e-3, 1e-1)
+    Vc, vs = _fp8_cache(B, N, d, 41, 0.5, 8.0)
+    for b in range(B):                                # per-sequence scale ranges
+        ks[b] *= 3.0 ** b
+        vs[b] *= 0.5 ** b
+    Qs = _rand((B, H, d), 42)
+    g = np.random.default_rng(43)
+    idx = np.full((B, n_idx), -1, dtype=np.int32)
+    for b in range(B - 1):
+        n = int(g.integers(5, n_idx + 1))
+        idx[b, :n] = np.sort(g.integers(0, N, size=n))     # repeats likely
+        idx[b, g.random(n_idx) < 0.2] = -1
+    idx[0, :3] = 17                                    # one key in three slots
+    idx[1, 5] = idx[1, 6] = 40
+    # sequence B-1: no valid slot -> zero output
+    scale = 1 / math.sqrt(d)
+    got = oracle.sparse_attn_decode(Qs, Kc, Vc, ks, vs, idx, range(B))
+    for b in range(B - 1):
+        assert np.allclose(got[b], _sparse_decode_ref(Qs, Kc, Vc, ks, vs, idx, b, scale), rtol=1e-12, atol=1e-12)
+    assert np.array_equal(got[B - 1], np.zeros((H, d)))
+    # planted mistakes in the gather, on the CPU: each moves some sequence's output far
+    swapped = oracle.sparse_attn_decode(Qs, Kc, Vc, vs, ks, idx, range(B - 1))
+    assert max(np.abs(swapped[b] - got[b]).max() for b in range(B - 1)) > 1e-2
+    shifted = oracle.sparse_attn_decode(Qs, torch.roll(Kc, 1, 0), torch.roll(Vc, 1, 0), ks, vs, idx, range(B - 1))
+    assert max(np.abs(shifted[b] - got[b]).max() for b in range(B - 1)) > 1e-2
+
+
+def test_sparse_row_with_no_valid_entry_is_zero():
+    q = _rand((4, 8), 44)
+    K = _rand((10, 8), 45)
+    V = _rand((10, 6), 46)
+    out = oracle.sparse_attn_row(q, K, V, np.full(5, -1, dtype=np.int32), 0.3)
+    assert out.shape == (4, 6) and np.array_equal(out, np.zeros((4, 6)))
+    # one valid entry: probability 1 on that key, the output is its V row
+    one = oracle.sparse_attn_row(q, K, V, np.array([-1, 7, -1], dtype=np.int32), 0.3)
+    assert np.allclose(one, np.broadcast_to(V[7], (4, 6)), rtol=0, atol=1e-15)
 
 
 def test_sparse_equals_dense_when_budget_covers_prefix():
