@@ -39,6 +39,7 @@ _MASK64 = (1 << 64) - 1
 STREAMS = {
     "q_full": 1, "k": 2, "v": 3, "needle": 4, "zipf": 5, "hidden": 6,
     "kv_scale_k": 7, "kv_scale_v": 8, "q_sparse": 100, "wk": 200, "wv": 300,
+    "q_bridged": 400,
 }
 
 
@@ -254,6 +255,18 @@ def make_bridge_case(R: int, D: int, d: int, n_layers: int, seed: int = 0,
     Wk = [normal_bf16(seed, STREAMS["wk"] + l, (d, D), ws, device) for l in range(n_layers)]
     Wv = [normal_bf16(seed, STREAMS["wv"] + l, (d, D), ws, device) for l in range(n_layers)]
     return BridgeCase(hidden, Wk, Wv)
+
+
+def bridged_decode_queries(B: int, H: int, d: int, n_layers: int, n_sparse: int, seed: int = 0,
+                           device="cpu") -> List[Tuple[torch.Tensor, List[torch.Tensor]]]:
+    """Per cross-decoder layer l: its full layer's new-token queries and those of
+    its n_sparse sparse layers, bf16 N(0,1) [B, H, d] (stream q_bridged + 10*l + i)."""
+    out = []
+    for l in range(n_layers):
+        base = STREAMS["q_bridged"] + 10 * l
+        q = normal_bf16(seed, base, (B, H, d), 1.0, device)
+        out.append((q, [normal_bf16(seed, base + 1 + i, (B, H, d), 1.0, device) for i in range(n_sparse)]))
+    return out
 
 
 # The five workloads (sizes from the method's own regimes: 32k pretraining,

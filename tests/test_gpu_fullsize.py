@@ -4,8 +4,9 @@ sampled rows / sequences that the fp64 oracle computes one by one.
 * prefill T = 32768, 16 heads, d = 256, N(0,1)/16 + 64 needles, 3 sparse layers
 * decode over an FP8 cache, 64 sequences x 131072 tokens, 3 sparse layers
 * chunked prefill T = 262144 (8192-query chunks), Zipf key norms, 2 sparse layers
-* bridged 1M decode: bridging of 4 x 2^20 hidden rows (2 layers) and decode of
-  4 sequences x 2^20 tokens over an FP8 cache
+* bridged 1M decode: bridging of 4 x 2^20 hidden rows into 2 layers' FP8
+  caches, then decode of 4 sequences x 2^20 tokens in both layers (full
+  attention + selection and 3 sparse layers each) over those bridged caches
 """
 import math
 
@@ -98,31 +99,38 @@ def test_prefill_256k_chunked_zipf(hs2):
         _select_and_sparse(hs2, case, rows, q_start=ci * ch, Tq=ch)
 
 
-def _decode_full(hs2, case, seqs):
-    B, N, H, d, W, k = case.B, case.N, case.H, case.d, case.window, case.topk
+def _decode_layer(hs2, Q, Q_sparse, Kc, Vc, ks, vs, B, N, H, d, W, k, seqs, cpu=None):
+    """Full layer (select) + its sparse layers over one FP8 cache, on the GPU,
+    checked against the oracle on the sequences ``seqs``; the sparse layers are
+    fed the oracle's index rows on those sequences (identical inputs)."""
     O = torch.empty(B, H, d, dtype=torch.bfloat16, device="cuda")
     idx = torch.empty(B, W + k, dtype=torch.int32, device="cuda")
     ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_FP8_E4M3, B, 1, N, H, d, W, k))
-    hs2.hs2_full_attn_select(case.Q, case.Kc, case.Vc, O, idx, ws, window=W, topk=k, k_scale=case.ks,
-                             v_scale=case.vs)
+    hs2.hs2_full_attn_select(Q, Kc, Vc, O, idx, ws, window=W, topk=k, k_scale=ks, v_scale=vs)
     assert hs2.hs2_device_status() == 0
     del ws
     oidx = idx.clone()
-    cpu = [t.cpu() for t in (case.Q, case.Kc, case.Vc, case.ks, case.vs)]
+    cpu = cpu or [t.cpu() for t in (Kc, Vc, ks, vs)]
+    Qc = Q.cpu()
     for b in seqs:
-        r = oracle.decode_select(*cpu, [b], N, W, k)[b]
+        r = oracle.decode_select(Qc, *cpu, [b], N, W, k)[b]
         ok, _, msg = check_idx_row(idx[b].cpu().numpy(), r, W, k)
         assert ok, msg
         assert max_abs(O[b].float().cpu().numpy(), r.O) <= TOL_FP8
         oidx[b] = torch.from_numpy(r.idx).cuda()
     wss = hs2.workspace(hs2.hs2_sparse_attn_decode_workspace(B, W + k, H, d))
-    for Qs in case.Q_sparse:
+    for Qs in Q_sparse:
         Os = torch.empty(B, H, d, dtype=torch.bfloat16, device="cuda")
-        hs2.hs2_sparse_attn_decode(Qs, case.Kc, case.Vc, case.ks, case.vs, oidx, Os, wss)
+        hs2.hs2_sparse_attn_decode(Qs, Kc, Vc, ks, vs, oidx, Os, wss)
         assert hs2.hs2_device_status() == 0
-        sref = oracle.sparse_attn_decode(Qs.cpu(), *cpu[1:], oidx.cpu(), seqs)
+        sref = oracle.sparse_attn_decode(Qs.cpu(), *cpu, oidx.cpu(), seqs)
         for b in seqs:
             assert max_abs(Os[b].float().cpu().numpy(), sref[b]) <= TOL_FP8
+
+
+def _decode_full(hs2, case, seqs):
+    _decode_layer(hs2, case.Q, case.Q_sparse, case.Kc, case.Vc, case.ks, case.vs, case.B, case.N, case.H,
+                  case.d, case.window, case.topk, seqs)
 
 
 def test_decode_64x128k_fp8(hs2):
@@ -133,11 +141,15 @@ def test_decode_64x128k_fp8(hs2):
 
 
 def test_bridged_decode_1m(hs2):
+    """Bridging of every token of the 4 sequences into the 2 cross-decoder
+    layers' FP8 caches (sampled rows against the oracle), then the decode step
+    of BOTH layers -- full attention + selection and 3 sparse layers each --
+    over those GPU-bridged caches, all 4 sequences against the oracle."""
     c = synth.CONFIGS[5]
-    B, N, D, d = c["B"], c["N"], c["D"], c["d"]
-    # bridging of every token of the 4 sequences into 2 layers' FP8 caches
+    B, N, D, d, H, W, k = c["B"], c["N"], c["D"], c["d"], c["H"], c["window"], c["topk"]
     bc = synth.make_bridge_case(B * N, D, d, c["n_layers"], seed=0, device="cuda")
     rows = _rows(B * N, 2048, 3, extra=[0, B * N - 1, N - 1, N])
+    caches = []
     for l in range(c["n_layers"]):
         K = torch.empty(B * N, d, dtype=torch.uint8, device="cuda")
         V = torch.empty_like(K)
@@ -146,14 +158,14 @@ def test_bridged_decode_1m(hs2):
         hs2.hs2_bridge_kv(bc.hidden, bc.Wk[l], bc.Wv[l], K, V, ks, vs)
         assert hs2.hs2_device_status() == 0
         hr = bc.hidden[rows].cpu()
-        for codes, sc, W in ((K, ks, bc.Wk[l]), (V, vs, bc.Wv[l])):
-            Wc = W.cpu()
+        for codes, sc, Wm in ((K, ks, bc.Wk[l]), (V, vs, bc.Wv[l])):
+            Wc = Wm.cpu()
             exact = oracle.bridge_rows(hr, Wc)
             sbad, bad = fp8_rule(codes[rows].cpu(), sc[rows].cpu(), exact, abs_dot(hr, Wc))
             assert sbad == 0 and bad == 0
-        del K, V, ks, vs
+        caches.append((K.view(B, N, d), V.view(B, N, d), ks.view(B, N), vs.view(B, N)))
     del bc
     torch.cuda.empty_cache()
-    # decode at 2^20 tokens over an FP8 cache from the input generator
-    case = synth.make_decode_case(B, N, c["H"], d, c["window"], c["topk"], c["n_sparse"], seed=5, device="cuda")
-    _decode_full(hs2, case, range(B))
+    queries = synth.bridged_decode_queries(B, H, d, c["n_layers"], c["n_sparse"], seed=0, device="cuda")
+    for (Kc, Vc, ks, vs), (Q, Qs) in zip(caches, queries):
+        _decode_layer(hs2, Q, Qs, Kc, Vc, ks, vs, B, N, H, d, W, k, range(B))

@@ -148,11 +148,14 @@ def test_sparse_decode_many_sequences(hs2):
     assert max(max_abs(O[b].float().numpy(), ref[b]) for b in range(B)) <= TOL_FP8
 
 
-@pytest.mark.parametrize("n_idx,H,d", [(1792, 16, 256), (2000, 16, 256), (1300, 8, 128), (5, 16, 256)])
+@pytest.mark.parametrize("n_idx,H,d", [(1920, 16, 256), (1793, 16, 256), (1792, 16, 256), (1920, 8, 128),
+                                       (1921, 16, 256), (2000, 16, 256), (1300, 8, 128), (5, 16, 256)])
 def test_sparse_prefill_index_widths(hs2, n_idx, H, d):
-    """Index rows at the tensor-core kernel's limit (14 tiles of 128 keys), past it (the
-    warp-pair kernel), a ragged H = 8, d = 128 case and a tiny one, each with empty (-1)
-    slots scattered through the row and repeated keys; sampled rows against the oracle."""
+    """Index rows at the tensor-core kernel's limit (15 tiles of 128 keys: 1920, and 1793,
+    the first width that needs the 15th tile), one tile below it, just past it (1921 and
+    2000: the warp-pair kernel), a ragged H = 8, d = 128 case and a tiny one, each with
+    empty (-1) slots scattered through the row and repeated keys; sampled rows against the
+    oracle."""
     T = 2200
     case = synth.make_prefill_case(T, H, d, 128, 64, n_sparse=1, seed=11)
     rng = np.random.default_rng(n_idx)
@@ -163,6 +166,64 @@ def test_sparse_prefill_index_widths(hs2, n_idx, H, d):
     rows = list(range(0, T, 173)) + [T - 1]
     ref = oracle.sparse_attn(case.Q_sparse[0], case.K, case.V, idx, rows)
     assert max(max_abs(O[t].float().numpy(), ref[t]) for t in rows) <= TOL_BF16
+
+
+def test_rows_with_no_valid_entry_give_zero(hs2):
+    """A row whose idx holds no valid entry selects nothing: its output is
+    exactly zero and nothing is reported, on the prefill kernel and on both
+    decode paths (a cluster per sequence at 70 sequences; split partials at 1)."""
+    T, H, d = 300, 16, 256
+    case = synth.make_prefill_case(T, H, d, 128, 64, n_sparse=1, seed=12)
+    idx = np.full((T, 192), -1, dtype=np.int32)
+    for t in range(T):
+        idx[t, :min(t + 1, 192)] = np.arange(max(0, t - 191), t + 1)
+    empty = [0, 7, 150, T - 1]
+    idx[empty] = -1
+    O = gpu_sparse_prefill(case.Q_sparse[0], case.K, case.V, idx)
+    for t in empty:
+        assert torch.count_nonzero(O[t]) == 0
+    rows = [1, 8, 151, 298]
+    ref = oracle.sparse_attn(case.Q_sparse[0], case.K, case.V, idx, rows)
+    assert max(max_abs(O[t].float().numpy(), ref[t]) for t in rows) <= TOL_BF16
+    for B in (70, 1, 3):
+        dc = synth.make_decode_case(B, 2000, 16, 256, 128, 1024, n_sparse=1, seed=13)
+        g = np.random.default_rng(B)
+        didx = np.sort(g.integers(0, 2000, size=(B, 1152)), axis=1).astype(np.int32)
+        gone = [0] if B == 1 else [0, B - 1]
+        didx[gone] = -1
+        Od = gpu_sparse_decode(dc, dc.Q_sparse[0], didx)
+        for b in gone:
+            assert torch.count_nonzero(Od[b]) == 0
+        live = [b for b in range(B) if b not in gone][:4]
+        if live:
+            dref = oracle.sparse_attn_decode(dc.Q_sparse[0], dc.Kc, dc.Vc, dc.ks, dc.vs, didx, live)
+            assert max(max_abs(Od[b].float().numpy(), dref[b]) for b in live) <= TOL_FP8
+
+
+@pytest.mark.parametrize("B,N", [(3, 5000), (70, 1500)])
+def test_decode_small_value_scales(hs2, B, N):
+    """A cache whose V scales are 2^-16 of the usual ones: every output is 2^-16
+    of the usual one.  The kernels hold p * v_scale in f16 against a per-row
+    power-of-two reference, so the result is the unscaled run's times 2^-16,
+    bit for bit, and the error relative to the output stays the unscaled one
+    (no f16 underflow), for the full layer and the sparse layer."""
+    case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=1, seed=14)
+    O1, idx1 = gpu_decode_select(case)
+    oidx = idx1.numpy()
+    Os1 = gpu_sparse_decode(case, case.Q_sparse[0], oidx)
+    small = synth.DecodeCase(case.B, case.N, case.H, case.d, case.window, case.topk, case.Q, case.Kc, case.Vc,
+                             case.ks, case.vs * 2.0 ** -16, case.Q_sparse)
+    O2, idx2 = gpu_decode_select(small)
+    Os2 = gpu_sparse_decode(small, small.Q_sparse[0], oidx)
+    assert torch.equal(idx1, idx2)
+    assert torch.equal(O2.float(), O1.float() * 2.0 ** -16)
+    assert torch.equal(Os2.float(), Os1.float() * 2.0 ** -16)
+    seqs = [0, B - 1]
+    ref = oracle.decode_select(small.Q, small.Kc, small.Vc, small.ks, small.vs, seqs, N, 128, 1024)
+    sref = oracle.sparse_attn_decode(small.Q_sparse[0], small.Kc, small.Vc, small.ks, small.vs, oidx, seqs)
+    for b in seqs:
+        for got, want in ((O2[b], ref[b].O), (Os2[b], sref[b])):
+            assert max_abs(got.float().numpy(), want) <= TOL_FP8 * 2.0 ** -16
 
 
 # ---------------------------------------------------------------- checks and faults

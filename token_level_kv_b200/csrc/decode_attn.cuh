@@ -8,10 +8,12 @@
 // Key j of sequence b is E4M3(K[b,j,:]) * k_scale[b,j], likewise V.
 //
 // Design (sm_100a), HBM-bound: everything serves bytes in flight.
-//   * One producer warp streams 16-key chunks into a shared ring of NS stages,
-//     so almost the whole ring is in flight whatever the consumers are doing;
-//     NC consumer warps take chunk i from stage i % NS (consumer i % NC) and
-//     hand the stage back through its empty barrier.  A range (a7) is
+//   * Producer warps stream 32-key chunks into a shared ring of NS stages,
+//     so almost the whole ring is in flight whatever the consumers are doing
+//     (one warp for a range, three for a gather, which needs a copy
+//     instruction per two rows); the consumer warp pairs take chunk i from
+//     stage i % NS (pair i % NP) and hand the stage back through its empty
+//     barrier.  A range (a7) is
 //     contiguous in the cache: one elected lane moves each chunk's K and V
 //     with 3-D TMA tiles (box 128 bytes x 16 keys, 128-byte swizzle; keys past
 //     kv_len arrive as zeros), which keeps the whole copy off the load/store
@@ -26,8 +28,11 @@
 //     prescale that puts its largest element in [2^14, 2^15) (f16 then holds
 //     every bf16 element exactly except ones below 2^-28 of that maximum);
 //     the prescale, the key scale and softmax_scale multiply the fp32 logit.
-//     P holds p * v_scale in f16 (p <= 2^8), so dequantised values must stay
-//     below the f16 maximum (|v| <= 65504), which real caches do.
+//     P holds p * v_scale * 2^-e in f16, e the exponent of the largest V scale
+//     a pair has seen (raised with an exact power-of-two rescale of O when a
+//     chunk brings a larger one, and undone when the pairs merge), so P stays
+//     below 2^9 (p <= 2^8) and neither overflows nor underflows whatever the
+//     magnitude of the scales: the result scales exactly with them.
 //   * S = Q K^T traverses the head dimension in a fixed permutation shared by
 //     Q and K (within each block of 16: thread t's k pairs {2t,2t+1} and
 //     {2t+8,2t+9} are the dims 4t..4t+3), so a thread's K fragment is ONE
@@ -66,10 +71,16 @@ namespace cg = cooperative_groups;
 
 template <int D, bool RANGE>
 struct DecLayout {
-  static constexpr int NP = 5;                      // consumer warp pairs
+  // A range moves each stage with one TMA instruction per box, so one
+  // producer warp keeps the ring full; a gather issues a copy instruction per
+  // two rows, and one warp could not issue them fast enough (measured: 1.6x
+  // slower than the random-row gather rate of the memory), so three warps
+  // share it.
+  static constexpr int NP = RANGE ? 5 : 4;          // consumer warp pairs
   static constexpr int NC = 2 * NP;                 // consumer warps
+  static constexpr int NPROD = RANGE ? 1 : 3;       // producer warps
   static constexpr int HD = D / 2;                  // dims per consumer warp
-  static constexpr int NT = (NC + 1) * 32;          // + one producer warp (11 warps: <= 168 registers)
+  static constexpr int NT = (NC + NPROD) * 32;      // 11 warps: <= 168 registers
   static constexpr int NS = 10;                     // ring stages (32 keys each)
   static constexpr int CH = 32;
   // gather stage: K rows, V rows at a padded stride, then the two scale rows
@@ -100,6 +111,8 @@ struct DecLayout {
                  : reinterpret_cast<float*>(smem + OFF_RING + s * STAGE + 2 * CH * (D + 16));
   }
 };
+
+constexpr int kNoVexp = -1000;   // no V scale seen yet
 
 struct DecParams {
   const __nv_bfloat16* Q;   // [B, H, D]
@@ -181,7 +194,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  __shared__ float red_max[L::NC + 1];
+  __shared__ float red_max[L::NC + L::NPROD];
   if (lane == 0) red_max[warp] = mx;
   cp_async_wait<0>();
   if (!RANGE) {
@@ -248,16 +261,20 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
     return true;
   };
+  // producer warp pw issues chunks pw, pw + NPROD, ... in increasing order;
+  // a chunk's slot waits only for the chunk NS before it, which some producer
+  // issues first, so the producers never wait on each other in a cycle
   const int first_round = min(n_chunks, L::NS);
+  const int pw = warp - L::NC;
   bool prod_ok = true;
-  int issued = 0;
-  if (warp == L::NC) {
+  int issued = pw;                                   // next chunk of this producer
+  if (warp >= L::NC) {
     if (RANGE && lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
     while (issued < first_round && prod_ok)
-      if ((prod_ok = produce(issued))) ++issued;
+      if ((prod_ok = produce(issued))) issued += L::NPROD;
   }
 
   float o[L::HD / 8][4];
@@ -265,11 +282,12 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   for (int i = 0; i < L::HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float qscale_inv = 1.f;
+  float vinv = 1.f;
   // ---- Q -> f16 with an exact power-of-two prescale (largest element in
   // [2^14, 2^15)), written while the first chunks are in flight
   {
     float m = 0.f;
-    for (int w = 0; w <= L::NC; ++w) m = fmaxf(m, red_max[w]);
+    for (int w = 0; w < L::NC + L::NPROD; ++w) m = fmaxf(m, red_max[w]);
     const int ex = m > 0.f ? 14 - ilogbf(m) : 0;
     const float qs = ldexpf(1.f, ex);
     qscale_inv = ldexpf(1.f, -ex);
@@ -293,10 +311,12 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   }
   __syncthreads();                                   // Q in shared memory
 
-  if (warp == L::NC) {
+  int vexp = kNoVexp;                                // power-of-two reference of the V scales (consumers)
+  if (warp >= L::NC) {
     while (issued < n_chunks && prod_ok)
-      if ((prod_ok = produce(issued))) ++issued;
+      if ((prod_ok = produce(issued))) issued += L::NPROD;
     asm volatile("cp.async.wait_all;" ::: "memory");  // every issued copy lands before the merge reuses the ring
+    static_assert(!RANGE || L::NPROD == 1, "the TMA drain below walks one producer's chunks");
     if (RANGE && lane == 0)                           // and every TMA tile (already done unless a wait gave up)
       for (int i = max(0, issued - L::NS); i < issued; ++i) mbar_drain(&full[i % L::NS], (uint32_t)((i / L::NS) & 1));
   } else {
@@ -421,6 +441,29 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
       }
       const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
       const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
+      // P enters the f16 product as p * v_scale * 2^-vexp, vexp the exponent
+      // of the largest V scale seen so far (raised, with an exact rescale of
+      // O, when a stage brings a larger one): p <= 2^8 keeps it below 2^9,
+      // and it no longer underflows when the scales themselves are small
+      float vmx = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) vmx = fmaxf(vmx, svs[(j >> 1) * 8 + 2 * t + (j & 1)]);
+      vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, 1));
+      vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, 2));
+      if (vmx > 0.f) {
+        const int ev = (int)((__float_as_uint(vmx) >> 23) & 0xffu) - 127;   // floor(log2) of a normal scale
+        if (ev > vexp) {
+          if (vexp != kNoVexp) {
+            const float r = ldexpf(1.f, vexp - ev);
+#pragma unroll
+            for (int j = 0; j < L::HD / 8; ++j) {
+              o[j][0] *= r; o[j][1] *= r; o[j][2] *= r; o[j][3] *= r;
+            }
+          }
+          vexp = ev;
+          vinv = ldexpf(1.f, -ev);
+        }
+      }
       float pv[4][4];
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
@@ -429,7 +472,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
         for (int e = 0; e < 4; ++e) {
           const float pe = fast_exp2(x[nt][e] - (e < 2 ? mu0 : mu1));
           if (e < 2) ls0 += pe; else ls1 += pe;
-          pv[nt][e] = pe * svs[nt * 8 + 2 * t + (e & 1)];
+          pv[nt][e] = pe * (svs[nt * 8 + 2 * t + (e & 1)] * vinv);
         }
       l0 = l0 * al0 + ls0;
       l1 = l1 * al1 + ls1;
@@ -481,6 +524,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   __syncthreads();
+  __shared__ int pexp[L::NP];
   float* cmb = reinterpret_cast<float*>(smem + L::Q_BYTES);    // [NP pairs] partials, O rows padded
   float* mine = cmb + L::NP * (L::PPART / 4);                   // merged partial of the CTA
   if (warp < L::NC) {
@@ -491,6 +535,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
       wpart[g + 8] = m1;
       wpart[16 + g] = l0;
       wpart[16 + g + 8] = l1;
+      if (g == 0) pexp[pr] = vexp == kNoVexp ? 0 : vexp;
     }
     // n-tiles 2q and 2q+1 (q = 2*b2 + half) hold, for rows g and g+8, the four
     // consecutive dims c0 + 4t .. c0 + 4t + 3 (c0 = hf*HD + 16q): one float4 each
@@ -503,7 +548,8 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
           make_float4(o[2 * q][2], o[2 * q + 1][2], o[2 * q][3], o[2 * q + 1][3]);
     }
   }
-  // per-head merge factors of the pairs, once: fac[w][h] = 2^(m_w - M_h)
+  // per-head merge factors of the pairs, once: fac[w][h] = 2^(m_w - M_h) for
+  // l, times 2^vexp_w for O (undoing the pair's V-scale reference)
   __shared__ float fac[L::NP][16];
   __shared__ float cfac[8][16];
   __shared__ float cinv[16];
@@ -516,7 +562,7 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
     for (int w = 0; w < L::NP; ++w) {
       const float mw = cmb[w * (L::PPART / 4) + h];
       const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-      fac[w][h] = f;
+      fac[w][h] = f * ldexpf(1.f, pexp[w]);
       Ls += cmb[w * (L::PPART / 4) + 16 + h] * f;
     }
     float* dst = PARTIALS ? p.part + ((int64_t)b * p.splits + split) * (32 + 16 * D) : mine;

@@ -587,11 +587,15 @@ hs2_status hs2_sparse_attn_decode_workspace(int batch, int n_idx, int Hq, int d,
   return HS2_OK;
 }
 
-hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
-                                  const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
-                                  int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
-                                  float softmax_scale, void* O, void* workspace, size_t ws_bytes, void* stream) {
-  g_err[0] = 0;
+}  // extern "C"
+
+namespace hs2 {
+namespace {
+// Argument checks of the sparse decode (with or without a caller workspace).
+hs2_status sparse_decode_args(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                              const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                              int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
+                              float softmax_scale, const void* O) {
   HS2_CHECK(Q && Kc && Vc && k_scale && v_scale && idx && O, HS2_ERR_INVALID_ARG, "null tensor pointer");
   HS2_CHECK(aligned16(Q) && aligned16(Kc) && aligned16(Vc) && aligned16(O) && aligned4(idx) && aligned4(k_scale) &&
                 aligned4(v_scale),
@@ -602,8 +606,23 @@ hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
   HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
   HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
   HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  return HS2_OK;
+}
+}  // namespace
+}  // namespace hs2
+
+extern "C" {
+
+hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                                  const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t kv_len,
+                                  int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
+                                  float softmax_scale, void* O, void* workspace, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  hs2_status s = sparse_decode_args(Q, Kc, Vc, k_scale, v_scale, kv_dtype, batch, kv_len, kv_stride_tokens, idx,
+                                    n_idx, Hq, d, softmax_scale, O);
+  if (s != HS2_OK) return s;
   size_t need = 0;
-  hs2_status s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need);
+  s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need);
   if (s != HS2_OK) return s;
   HS2_CHECK(ws_bytes >= need && (need == 0 || (workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0))),
             HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
@@ -673,9 +692,11 @@ hs2_status hs2_sparse_attn_decode_static(const void* Q, const void* Kc, const vo
                                          int64_t kv_stride_tokens, const int32_t* idx, int n_idx, int Hq, int d,
                                          float softmax_scale, void* O, void* stream) {
   g_err[0] = 0;
-  size_t need = 0;
-  hs2_status s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need);
+  hs2_status s = sparse_decode_args(Q, Kc, Vc, k_scale, v_scale, kv_dtype, batch, kv_len, kv_stride_tokens, idx,
+                                    n_idx, Hq, d, softmax_scale, O);
   if (s != HS2_OK) return s;
+  size_t need = 0;
+  if ((s = hs2_sparse_attn_decode_workspace(batch, n_idx, Hq, d, &need)) != HS2_OK) return s;
   HS2_CHECK(need <= HS2_STATIC_SCRATCH_BYTES, HS2_ERR_UNSUPPORTED,
             "this batch needs %zu bytes of split scratch; the static array holds %u "
             "(use hs2_sparse_attn_decode with a workspace)", need, (unsigned)HS2_STATIC_SCRATCH_BYTES);
