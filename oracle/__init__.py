@@ -175,6 +175,64 @@ def select_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, p: int, window: int,
     return SelectRow(p, O, m, l, sigma, idx, tau, int(sel.shape[0]))
 
 
+@dataclass
+class BlockSelectRow:
+    p: int
+    sigma: np.ndarray         # [p+1] head-summed probabilities
+    block_score: np.ndarray   # [n_blocks] sum of sigma over each block's candidates
+    blocks: np.ndarray        # selected block numbers, ascending
+    idx: np.ndarray           # [window + topk_blocks * block] int32
+    tau: Optional[float]      # k-th largest block score (None: all blocks taken)
+
+
+def block_select_row(sigma: np.ndarray, p: int, window: int, block: int,
+                     topk_blocks: int) -> BlockSelectRow:
+    """Block-level selection (the ablation's alternative to token level).
+
+    The pages compare token-level selection with block-level selection of
+    64-token blocks at the same 1024-token budget (agihunt.info summary,
+    ablation paragraph; 10100.com article, "evolution one": blocks of 64 or
+    128 tokens).  Readings: blocks are aligned, block c = positions
+    [c*block, (c+1)*block); a block's score is the sum of sigma over its
+    out-of-window candidates (positions <= p - window), so the boundary block
+    counts only those; the topk_blocks blocks with the largest score are taken
+    (ties to the smaller block number, all of them if there are fewer), and the
+    index row is the forced window, then every candidate position of the
+    selected blocks ascending, then -1.
+    """
+    n_cand = max(0, p - window + 1)
+    nb = (n_cand + block - 1) // block
+    score = np.zeros(nb, dtype=np.float64)
+    for c in range(nb):
+        score[c] = sigma[c * block:min(n_cand, (c + 1) * block)].sum()
+    chosen = topk_positions(score, topk_blocks)            # same rule as tokens
+    tau = None
+    if nb > topk_blocks:
+        tau = float(np.sort(score)[-topk_blocks])
+    idx = np.full(window + topk_blocks * block, -1, dtype=np.int32)
+    idx[:window] = window_slots(p, window)
+    pos = [j for c in chosen for j in range(c * block, min(n_cand, (c + 1) * block))]
+    idx[window:window + len(pos)] = pos
+    return BlockSelectRow(p, sigma, score, np.asarray(chosen, dtype=np.int64), idx, tau)
+
+
+def full_attn_select_blocks(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rows: Sequence[int],
+                            q_start: int, window: int, block: int, topk_blocks: int,
+                            scale: Optional[float] = None):
+    """The full layer with block-level selection: per row the token-level
+    SelectRow (its O, m, l, sigma; the token index set is not used) and the
+    BlockSelectRow built from the same sigma."""
+    d = Q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    K = f64(K)
+    V = f64(V)
+    out = {}
+    for t in rows:
+        r = select_row(f64(Q[t]), K, V, q_start + t, window, 1, scale)
+        out[t] = (r, block_select_row(r.sigma, q_start + t, window, block, topk_blocks))
+    return out
+
+
 def full_attn_select(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rows: Sequence[int],
                      q_start: int, window: int, topk: int,
                      scale: Optional[float] = None) -> Dict[int, SelectRow]:

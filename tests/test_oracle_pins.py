@@ -426,3 +426,61 @@ def test_pins_catch_a_shifted_window():
     assert good[-1] == p and good[0] == p - W + 1
     shifted = oracle.window_slots(p - 1, W)
     assert not np.array_equal(shifted, good)
+
+
+# ---------------------------------------------------------------- block-level selection
+
+def test_block_selection_with_block_1_is_token_selection():
+    """Blocks of one token are tokens: the block variant's index rows equal the
+    token-level rows for every query (same k), which are pinned above."""
+    T, H, d, W, k = 120, 4, 16, 8, 9
+    q, K, V = _rand((T, H, d), 700), _rand((T, d), 701), _rand((T, d), 702)
+    tok = oracle.full_attn_select(q, K, V, range(T), 0, W, k)
+    blk = oracle.full_attn_select_blocks(q, K, V, range(T), 0, W, 1, k)
+    for t in range(T):
+        assert np.array_equal(blk[t][1].idx, tok[t].idx)
+        assert blk[t][1].tau == tok[t].tau
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_block_selection_brute_force_tiny(seed):
+    """Every k-subset of blocks on rows of up to 40 candidates: the chosen
+    blocks are the unique subset that outranks the rest under (score, -block);
+    the row lists exactly their candidate positions; the scores partition the
+    candidates' sigma."""
+    T, H, d, W, B, k = 48, 3, 4, 4, 4, 3
+    q, K = _rand((T, H, d), 800 + seed), _rand((T, d), 810 + seed)
+    if seed % 2:
+        K[4:8] = K[12:16]                          # two blocks with equal scores where sigma allows
+    rows = oracle.full_attn_select_blocks(q, K, _rand((T, d), 820 + seed), range(T), 0, W, B, k)
+    for t, (r, b) in rows.items():
+        n_cand = max(0, t - W + 1)
+        nb = (n_cand + B - 1) // B
+        assert b.block_score.shape == (nb,)
+        assert abs(b.block_score.sum() - r.sigma[:n_cand].sum()) <= 1e-12
+        ref = _brute_force_topk(b.block_score, k)
+        assert tuple(b.blocks.tolist()) == ref
+        want = [j for c in ref for j in range(c * B, min(n_cand, (c + 1) * B))]
+        n = len(want)
+        assert list(b.idx[W:W + n]) == want and np.all(b.idx[W + n:] == -1)
+        assert np.array_equal(b.idx[:W], oracle.window_slots(t, W))
+        if nb > k:
+            assert b.tau == float(torch.topk(torch.from_numpy(b.block_score), k).values[-1])
+
+
+def test_block_selection_uniform_closed_form():
+    """K = 0: sigma = H/(p+1) for every key, so every full block scores
+    B*H/(p+1), the partial boundary block less, and with the full blocks tied
+    the selection is the first k blocks."""
+    T, H, d, W, B, k = 200, 4, 8, 16, 8, 5
+    rows = oracle.full_attn_select_blocks(_rand((T, H, d), 830), np.zeros((T, d)), _rand((T, d), 831),
+                                          range(T), 0, W, B, k)
+    for t, (r, b) in rows.items():
+        n_cand = max(0, t - W + 1)
+        full = n_cand // B
+        assert np.allclose(b.block_score[:full], B * H / (t + 1), rtol=1e-13)
+        if n_cand % B:
+            assert np.isclose(b.block_score[-1], (n_cand % B) * H / (t + 1), rtol=1e-13)
+        nb = b.block_score.shape[0]
+        expect = list(range(min(k, nb))) if full >= k or nb <= k else list(range(full)) + [nb - 1]
+        assert b.blocks.tolist() == expect
