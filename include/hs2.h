@@ -38,7 +38,7 @@
  *   - No exception or abort crosses the ABI.  Calls on distinct workspaces may
  *     run concurrently from several host threads.
  *   - Supported in this version: one KV head, Hq in {8, 16}, d in {128, 256},
- *     window + topk <= 2048, window >= 1.
+ *     index rows (window + selection) of at most 2048 entries, window >= 1.
  */
 #ifndef HS2_H_
 #define HS2_H_
@@ -98,6 +98,29 @@ HS2_API hs2_status hs2_bridge_kv(const void* hidden, int64_t rows, int hidden_di
                          void* stream);
 
 /*
+ * Decode-step KV Bridging: append each sequence's new token to this layer's
+ * FP8 cache (agihunt.info summary, KV Bridging paragraph; arXiv abstract --
+ * every cross-decoder KV cache is built from self-decoder hidden states, so
+ * each decode step bridges the new token's hidden row).  For b < batch:
+ *     k = hidden[b,:] Wk^T,  v = hidden[b,:] Wv^T      (fp32 accumulation)
+ *     k_scale[b,pos[b]] = amax(k)/448 (1 if k is all zero)
+ *     Kc[b,pos[b],:]    = E4M3_RNE_satfinite(k / k_scale[b,pos[b]])   (V likewise)
+ * the same arithmetic as hs2_bridge_kv's FP8 output, one row per sequence.
+ *   hidden : bf16 [batch, hidden_dim] (the new tokens' self-decoder hidden states)
+ *   Wk, Wv : bf16 [d, hidden_dim]
+ *   Kc, Vc : uint8 [batch, kv_stride_tokens, d]; k_scale, v_scale fp32 [batch, kv_stride_tokens]
+ *   pos    : int32 [batch] on the device, the row written in each sequence.
+ * Only row pos[b] of each sequence is written.  An entry pos[b] outside
+ * [0, kv_stride_tokens) is skipped and raises HS2_ERR_DEVICE_CHECK in
+ * hs2_device_status().  Requires 1 <= batch <= 65535, hidden_dim a positive
+ * multiple of 256, d == 256.
+ */
+HS2_API hs2_status hs2_bridge_append(const void* hidden, int batch, int hidden_dim, const void* Wk,
+                                     const void* Wv, int d, void* Kc, void* Vc, float* k_scale,
+                                     float* v_scale, int64_t kv_stride_tokens, const int32_t* pos,
+                                     void* stream);
+
+/*
  * Full-attention layer as the oracle selector (agihunt.info summary, KV Reuse
  * and MQA/NoPE paragraphs).  Query t of sequence b sits at absolute position
  * p = q_start + t and attends causally to keys 0..p of its sequence:
@@ -128,6 +151,31 @@ HS2_API hs2_status hs2_full_attn_select(const void* Q, const void* K, const void
                                 int Hq, int d, int window, int topk, float softmax_scale,
                                 void* O, int32_t* idx, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/*
+ * The same full-attention layer with BLOCK-level selection, the alternative
+ * the pages measure token-level selection against (agihunt.info summary,
+ * ablation paragraph: 64-token blocks at the same 1024-token budget; 10100.com
+ * article, "evolution one").  Blocks are aligned: block c holds positions
+ * [c*block, (c+1)*block).  Block c's score is the sum of sigma_j over its
+ * candidates j <= p-window (the boundary block counts only those):
+ *     idx[b,t,0:window]  = p-window+1 .. p (-1 where negative)
+ *     idx[b,t,window:]   = every candidate position of the topk_blocks blocks
+ *                          with the largest score (ties to the smaller block;
+ *                          all blocks if there are at most topk_blocks),
+ *                          ascending, then -1 up to window + topk_blocks*block.
+ * Arguments, outputs, workspace (the same query, with topk = topk_blocks) and
+ * errors as hs2_full_attn_select; O is the same full-attention output.
+ * Requires block a power of two in [16, 256], window + topk_blocks*block <=
+ * 2048 and at most 16384 candidate blocks per query.
+ */
+HS2_API hs2_status hs2_full_attn_select_blocks(const void* Q, const void* K, const void* V,
+                                       const float* k_scale, const float* v_scale,
+                                       hs2_kv_dtype kv_dtype, int batch, int64_t q_start,
+                                       int64_t Tq, int64_t kv_len, int64_t kv_stride_tokens, int Hq,
+                                       int d, int window, int block, int topk_blocks,
+                                       float softmax_scale, void* O, int32_t* idx, void* workspace,
+                                       size_t ws_bytes, void* stream);
 
 /* Workspace bytes hs2_full_attn_select needs for these shape arguments. */
 HS2_API hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int64_t Tq,

@@ -58,3 +58,47 @@ def max_abs(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.max(np.abs(a - b))) if a.size else 0.0
+
+
+def check_block_row(gpu_row, ora_blk, window: int, block: int, topk_blocks: int, rel: float = TIE_REL):
+    """Block-level rows: window bit-exact; the selection is whole candidate
+    blocks (each block's candidate positions, consecutive), ascending, then -1;
+    the chosen block set equals the oracle's except for blocks whose score lies
+    within ``rel`` of the oracle's k-th largest block score.  ``ora_blk`` is an
+    oracle BlockSelectRow.  Returns (ok, n_swaps, message)."""
+    g = np.asarray(gpu_row).astype(np.int64)
+    o = ora_blk.idx.astype(np.int64)
+    p = ora_blk.p
+    if g.shape != o.shape:
+        return False, 0, f"shape {g.shape} vs {o.shape}"
+    if not np.array_equal(g[:window], o[:window]):
+        return False, 0, f"window segment differs at p={p}"
+    sel = g[window:]
+    n = int((sel >= 0).sum())
+    if not np.all(sel[:n] >= 0) or not np.all(sel[n:] == -1):
+        return False, 0, f"p={p}: selection not packed then -1 padded"
+    n_cand = max(0, p - window + 1)
+    blocks = []
+    i = 0
+    while i < n:
+        c = int(sel[i] // block)
+        want = np.arange(c * block, min(n_cand, (c + 1) * block))
+        if want.size == 0 or not np.array_equal(sel[i:i + want.size], want):
+            return False, 0, f"p={p}: block {c} not emitted whole at slot {i}"
+        if blocks and c <= blocks[-1]:
+            return False, 0, f"p={p}: blocks not ascending"
+        blocks.append(c)
+        i += want.size
+    nb = ora_blk.block_score.shape[0]
+    if len(blocks) != min(topk_blocks, nb):
+        return False, 0, f"p={p}: {len(blocks)} blocks vs {min(topk_blocks, nb)}"
+    diff = set(blocks) ^ set(ora_blk.blocks.tolist())
+    if not diff:
+        return True, 0, ""
+    if ora_blk.tau is None:
+        return False, len(diff), f"p={p}: all blocks must be taken"
+    for c in diff:
+        if abs(ora_blk.block_score[c] - ora_blk.tau) > rel * ora_blk.tau:
+            return False, len(diff), (f"p={p}: block {c} score={ora_blk.block_score[c]:.10g} "
+                                      f"tau={ora_blk.tau:.10g} outside the tie margin")
+    return True, len(diff) // 2, ""

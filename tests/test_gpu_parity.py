@@ -14,7 +14,7 @@ import oracle
 import synth
 from hs2_cases import (abs_dot, bf16_rule, check_select_rows, fp8_rule, gpu_decode_select, gpu_prefill_select,
                        gpu_sparse_decode, gpu_sparse_prefill)
-from parity import TOL_BF16, TOL_FP8, check_idx_row, max_abs
+from parity import TOL_BF16, TOL_FP8, check_block_row, check_idx_row, max_abs
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +59,41 @@ def test_bridge_fp8(hs2, rows):
         sbad, bad = fp8_rule(codes.cpu()[nz], sc.cpu()[nz], exact[nz], abs_dot(c.hidden, W)[nz])
         assert sbad == 0, f"{sbad} row scales off by more than the accumulation bound"
         assert bad == 0, f"{bad} FP8 codes off by more than the rounding rule"
+
+
+def test_bridge_append_writes_one_fp8_row_per_sequence(hs2):
+    """Decode-step bridging: each sequence's new hidden row is projected and its
+    FP8 K/V row and scales written at pos[b]; every other cache byte is left
+    as it was; an out-of-range pos is reported and skipped."""
+    B, S, D, d = 6, 300, 2048, 256
+    c = synth.make_bridge_case(B, D, d, 1, seed=15)
+    c.hidden[3] = 0                       # all-zero row: codes 0, scale 1
+    g = torch.Generator().manual_seed(0)
+    Kc = torch.randint(0, 255, (B, S, d), dtype=torch.uint8, generator=g)
+    Vc = torch.randint(0, 255, (B, S, d), dtype=torch.uint8, generator=g)
+    ks = torch.rand(B, S, generator=g)
+    vs = torch.rand(B, S, generator=g)
+    pos = torch.tensor([0, 17, 299, 5, 100, 299], dtype=torch.int32)
+    dev = [t.cuda() for t in (Kc, Vc, ks, vs)]
+    hs2.hs2_bridge_append(c.hidden.cuda(), c.Wk[0].cuda(), c.Wv[0].cuda(), *dev, pos.cuda())
+    assert hs2.hs2_device_status() == 0
+    Kg, Vg, ksg, vsg = (t.cpu() for t in dev)
+    rows = torch.arange(B)
+    for got, before, sc, sc_before, W in ((Kg, Kc, ksg, ks, c.Wk[0]), (Vg, Vc, vsg, vs, c.Wv[0])):
+        mask = torch.ones(B, S, dtype=torch.bool)
+        mask[rows, pos.long()] = False
+        assert torch.equal(got[mask], before[mask]) and torch.equal(sc[mask], sc_before[mask])
+        codes, scales = got[rows, pos.long()], sc[rows, pos.long()]
+        exact = oracle.bridge_rows(c.hidden, W)
+        assert float(scales[3]) == 1.0 and int(codes[3].sum()) == 0
+        nz = np.abs(exact).max(1) > 0
+        sbad, bad = fp8_rule(codes[nz], scales[nz], exact[nz], abs_dot(c.hidden, W)[nz])
+        assert sbad == 0 and bad == 0
+    bad_pos = pos.clone()
+    bad_pos[2] = S                        # one row past the cache
+    hs2.hs2_bridge_append(c.hidden.cuda(), c.Wk[0].cuda(), c.Wv[0].cuda(), *dev, bad_pos.cuda())
+    assert hs2.hs2_device_status() == 6   # HS2_ERR_DEVICE_CHECK, and nothing written for it
+    assert torch.equal(dev[0][2].cpu(), Kg[2])
 
 
 # ---------------------------------------------------------------- prefill select
@@ -114,6 +149,49 @@ def test_chunked_prefill_equals_one_call(hs2):
     assert torch.equal(torch.cat([idxa, idxb]), idx1)
     assert torch.equal(torch.cat([Oa, Ob]), O1)
     check_select_rows(case, Ob, idxb, [0, 1, 500, 895], q_start=904)
+
+
+@pytest.mark.parametrize("T,H,d,W,B,k,scale", [(2600, 16, 256, 128, 64, 16, 1 / 16), (1500, 8, 128, 128, 32, 8, 1.0),
+                                                (700, 16, 256, 64, 256, 4, 1.0), (900, 16, 128, 32, 16, 40, 1.0),
+                                                (300, 16, 256, 128, 64, 16, 1.0)])
+def test_prefill_block_selection(hs2, T, H, d, W, B, k, scale):
+    """Block-level selection on the GPU against the oracle: whole blocks, the
+    block set within the tie margin, the same full-attention output; rows with
+    fewer candidate blocks than k (all taken), a partial boundary block, near
+    uniform attention (scale 1/16) and several block sizes."""
+    case = synth.make_prefill_case(T, H, d, W, k * B, n_sparse=0, scale=scale, seed=16)
+    Q, K, V = case.Q.cuda(), case.K.cuda(), case.V.cuda()
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(T, W + k * B, dtype=torch.int32, device="cuda")
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_BF16, 1, T, T, H, d, W, k))
+    hs2.hs2_full_attn_select_blocks(Q, K, V, O, idx, ws, window=W, block=B, topk_blocks=k)
+    assert hs2.hs2_device_status() == 0
+    rows = sorted(set(list(range(0, T, 37)) + [W - 1, W, W + B - 1, W + B, W + k * B, T - 1]) & set(range(T)))
+    ref = oracle.full_attn_select_blocks(case.Q, case.K, case.V, rows, 0, W, B, k)
+    idx_c, O_c = idx.cpu().numpy(), O.float().cpu().numpy()
+    for t in rows:
+        r, b = ref[t]
+        ok, _, msg = check_block_row(idx_c[t], b, W, B, k)
+        assert ok, msg
+        assert max_abs(O_c[t], r.O) <= TOL_BF16
+
+
+def test_decode_block_selection_fp8(hs2):
+    B, N, Bk, k = 3, 5000, 64, 16
+    case = synth.make_decode_case(B, N, 16, 256, 128, k * Bk, n_sparse=0, seed=17)
+    O = torch.empty(B, 16, 256, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(B, 128 + k * Bk, dtype=torch.int32, device="cuda")
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_FP8_E4M3, B, 1, N, 16, 256, 128, k))
+    dev = [t.cuda() for t in (case.Q, case.Kc, case.Vc, case.ks, case.vs)]
+    hs2.hs2_full_attn_select_blocks(dev[0], dev[1], dev[2], O, idx, ws, window=128, block=Bk, topk_blocks=k,
+                                    k_scale=dev[3], v_scale=dev[4])
+    assert hs2.hs2_device_status() == 0
+    ref = oracle.decode_select(case.Q, case.Kc, case.Vc, case.ks, case.vs, range(B), N, 128, 1)
+    for b in range(B):
+        blk = oracle.block_select_row(ref[b].sigma, N - 1, 128, Bk, k)
+        ok, _, msg = check_block_row(idx[b].cpu().numpy(), blk, 128, Bk, k)
+        assert ok, msg
+        assert max_abs(O[b].float().cpu().numpy(), ref[b].O) <= TOL_FP8
 
 
 # ---------------------------------------------------------------- decode

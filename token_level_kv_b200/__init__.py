@@ -42,7 +42,9 @@ def _load() -> ctypes.CDLL:
         "hs2_last_error": ([], ctypes.c_char_p),
         "hs2_version": ([], ctypes.c_char_p),
         "hs2_bridge_kv": ([P, L, I, P, P, I, I, P, P, P, P, P], I),
+        "hs2_bridge_append": ([P, I, I, P, P, I, P, P, P, P, L, P, P], I),
         "hs2_full_attn_select": ([P, P, P, P, P, I, I, L, L, L, L, I, I, I, I, F, P, P, P, Z, P], I),
+        "hs2_full_attn_select_blocks": ([P, P, P, P, P, I, I, L, L, L, L, I, I, I, I, I, F, P, P, P, Z, P], I),
         "hs2_full_attn_select_workspace": ([I, I, L, L, I, I, I, I, ctypes.POINTER(Z)], I),
         "hs2_sparse_attn_prefill": ([P, P, P, P, L, L, I, I, I, F, P, P], I),
         "hs2_sparse_attn_decode": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P, Z, P], I),
@@ -64,7 +66,8 @@ lib = _load()
 EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv", "hs2_full_attn_select",
            "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
            "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit",
-           "hs2_profile_enable", "hs2_profile_collect", "hs2_sparse_attn_decode_static")
+           "hs2_profile_enable", "hs2_profile_collect", "hs2_sparse_attn_decode_static", "hs2_bridge_append",
+           "hs2_full_attn_select_blocks")
 
 
 def _check(status: int) -> None:
@@ -111,6 +114,17 @@ def hs2_bridge_kv(hidden, Wk, Wv, K_out, V_out, k_scale=None, v_scale=None, stre
                              _ptr(k_scale), _ptr(v_scale), _stream(stream)))
 
 
+def hs2_bridge_append(hidden, Wk, Wv, Kc, Vc, k_scale, v_scale, pos, stream=None) -> None:
+    """Bridge each sequence's new token (hidden [B, D]) and write its FP8 K/V row
+    and scales at row pos[b] of the caches Kc, Vc [B, stride, d], k_scale, v_scale [B, stride]."""
+    B, D = hidden.shape
+    d = Wk.shape[0]
+    if Kc.dim() != 3 or Kc.shape[0] != B or k_scale.shape != Kc.shape[:2]:
+        raise ValueError("caches must be [B, stride, d] with scales [B, stride]")
+    _check(lib.hs2_bridge_append(_ptr(hidden), B, D, _ptr(Wk), _ptr(Wv), d, _ptr(Kc), _ptr(Vc), _ptr(k_scale),
+                                 _ptr(v_scale), Kc.shape[1], _ptr(pos), _stream(stream)))
+
+
 def hs2_full_attn_select_workspace(kv_dtype: int, batch: int, Tq: int, kv_len: int, Hq: int, d: int,
                                    window: int, topk: int) -> int:
     n = ctypes.c_size_t(0)
@@ -127,6 +141,25 @@ def hs2_full_attn_select(Q, K, V, O, idx, workspace, *, window: int, topk: int, 
     decode (FP8 K/V codes): Q [B, H, d], K/V [B, stride, d], k/v_scale [B, stride],
     O [B, H, d], idx [B, window+topk]; the query sits at kv_len - 1.
     """
+    a = _select_args(Q, K, q_start, kv_len, softmax_scale, workspace)
+    _check(lib.hs2_full_attn_select(_ptr(Q), _ptr(K), _ptr(V), _ptr(k_scale), _ptr(v_scale), a["kvd"], a["batch"],
+                                    a["q_start"], a["Tq"], a["kv_len"], a["stride"], a["H"], a["d"], window, topk,
+                                    a["scale"], _ptr(O), _ptr(idx), _ptr(workspace), a["ws"], _stream(stream)))
+
+
+def hs2_full_attn_select_blocks(Q, K, V, O, idx, workspace, *, window: int, block: int, topk_blocks: int,
+                                q_start: int = 0, kv_len: int | None = None, k_scale=None, v_scale=None,
+                                softmax_scale: float | None = None, stream=None) -> None:
+    """Full-attention layer + block-level selection: as hs2_full_attn_select with
+    idx [rows, window + topk_blocks * block] holding the chosen blocks' positions."""
+    a = _select_args(Q, K, q_start, kv_len, softmax_scale, workspace)
+    _check(lib.hs2_full_attn_select_blocks(_ptr(Q), _ptr(K), _ptr(V), _ptr(k_scale), _ptr(v_scale), a["kvd"],
+                                           a["batch"], a["q_start"], a["Tq"], a["kv_len"], a["stride"], a["H"], a["d"],
+                                           window, block, topk_blocks, a["scale"], _ptr(O), _ptr(idx),
+                                           _ptr(workspace), a["ws"], _stream(stream)))
+
+
+def _select_args(Q, K, q_start, kv_len, softmax_scale, workspace) -> dict:
     kvd = _kv_dtype(K)
     d = Q.shape[-1]
     H = Q.shape[-2]
@@ -141,9 +174,8 @@ def hs2_full_attn_select(Q, K, V, O, idx, workspace, *, window: int, topk: int, 
         kv_len = stride if kv_len is None else kv_len
         q_start = kv_len - 1
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.hs2_full_attn_select(_ptr(Q), _ptr(K), _ptr(V), _ptr(k_scale), _ptr(v_scale), kvd, batch,
-                                    q_start, Tq, kv_len, stride, H, d, window, topk, scale, _ptr(O), _ptr(idx),
-                                    _ptr(workspace), ws, _stream(stream)))
+    return dict(kvd=kvd, d=d, H=H, scale=scale, batch=batch, Tq=Tq, kv_len=kv_len, stride=stride, q_start=q_start,
+                ws=ws)
 
 
 def hs2_sparse_attn_prefill(Q, K, V, idx, O, *, kv_len: int | None = None, softmax_scale: float | None = None,

@@ -14,6 +14,8 @@
 #include <mutex>
 
 #include "attn16.cuh"
+#include "bridge_append.cuh"
+#include "block_select.cuh"
 #include "bridge_gemm.cuh"
 #include "common.cuh"
 #include "decode_attn.cuh"
@@ -289,9 +291,43 @@ hs2_status launch_decode_cluster(const DecParams& p, int batch, cudaStream_t st,
   return after_launch("decode_attn_kernel", st);
 }
 
+// The last stage of a full layer: top-k tokens (block == 0) or top-k blocks
+// of `block` tokens per row, from the selection scores in the workspace.
+hs2_status launch_select(const float* sigma, int64_t ld, int64_t p0, int64_t pstep, int window, int topk, int block,
+                         int32_t* idx, int64_t rows, cudaStream_t st, const DevCtx& ctx) {
+  hs2_status s;
+  if (block == 0) {
+    TopkParams tp;
+    tp.sigma = sigma;
+    tp.ld = ld;
+    tp.p0 = p0;
+    tp.pstep = pstep;
+    tp.window = window;
+    tp.topk = topk;
+    tp.idx = idx;
+    if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
+    prof_begin(st);
+    topk_select_kernel<<<(unsigned)rows, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
+    return after_launch("topk_select_kernel", st);
+  }
+  BlockSelParams bp;
+  bp.sigma = sigma;
+  bp.ld = ld;
+  bp.p0 = p0;
+  bp.pstep = pstep;
+  bp.window = window;
+  bp.block = block;
+  bp.topk_blocks = topk;
+  bp.idx = idx;
+  if ((s = set_smem(block_select_kernel, BS_SMEM)) != HS2_OK) return s;
+  prof_begin(st);
+  block_select_kernel<<<(unsigned)rows, BS_THREADS, BS_SMEM, st>>>(bp, ctx);
+  return after_launch("block_select_kernel", st);
+}
+
 template <int D>
 hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q_start, int64_t Tq, int64_t kv_len,
-                          int Hq, int window, int topk, float scale, void* O, int32_t* idx, void* ws,
+                          int Hq, int window, int topk, int block, float scale, void* O, int32_t* idx, void* ws,
                           cudaStream_t st, const DevCtx& ctx) {
   const PrefillWs w = prefill_ws(Tq, kv_len, Hq);
   float* ml = reinterpret_cast<float*>(ws);
@@ -339,25 +375,13 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
     select_sigma_kernel<D, 8><<<sp.n_groups, SG_THREADS, SgLayout<D>::SMEM, st>>>(mQ256, mK, sp, ctx);
   }
   if ((s = after_launch("select_sigma_kernel", st)) != HS2_OK) return s;
-
-  TopkParams tp;
-  tp.sigma = sigma;
-  tp.ld = w.ld;
-  tp.p0 = q_start;
-  tp.pstep = 1;
-  tp.window = window;
-  tp.topk = topk;
-  tp.idx = idx;
-  if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
-  prof_begin(st);
-  topk_select_kernel<<<(unsigned)Tq, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
-  return after_launch("topk_select_kernel", st);
+  return launch_select(sigma, w.ld, q_start, 1, window, topk, block, idx, Tq, st, ctx);
 }
 
 template <int D>
 hs2_status decode_select(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
-                         int64_t kv_len, int64_t kv_stride, int Hq, int window, int topk, float scale, void* O,
-                         int32_t* idx, void* ws, cudaStream_t st, const DevCtx& ctx) {
+                         int64_t kv_len, int64_t kv_stride, int Hq, int window, int topk, int block, float scale,
+                         void* O, int32_t* idx, void* ws, cudaStream_t st, const DevCtx& ctx) {
   const DecodeWs w = decode_ws(batch, kv_len, Hq, D);
   uint8_t* b = static_cast<uint8_t*>(ws);
   float* logits = reinterpret_cast<float*>(b);
@@ -401,18 +425,7 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
     decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld);
     if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
   }
-  TopkParams tp;
-  tp.sigma = sigma;
-  tp.ld = w.ld;
-  tp.p0 = kv_len - 1;
-  tp.pstep = 0;
-  tp.window = window;
-  tp.topk = topk;
-  tp.idx = idx;
-  if ((s = set_smem(topk_select_kernel, TK_SMEM)) != HS2_OK) return s;
-  prof_begin(st);
-  topk_select_kernel<<<(unsigned)batch, TK_THREADS, TK_SMEM, st>>>(tp, ctx);
-  return after_launch("topk_select_kernel", st);
+  return launch_select(sigma, w.ld, kv_len - 1, 0, window, topk, block, idx, batch, st, ctx);
 }
 
 }  // namespace
@@ -480,6 +493,38 @@ hs2_status hs2_bridge_kv(const void* hidden, int64_t rows, int hidden_dim, const
   return after_launch("bridge_gemm_kernel", static_cast<cudaStream_t>(stream));
 }
 
+hs2_status hs2_bridge_append(const void* hidden, int batch, int hidden_dim, const void* Wk, const void* Wv, int d,
+                             void* Kc, void* Vc, float* k_scale, float* v_scale, int64_t kv_stride_tokens,
+                             const int32_t* pos, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(hidden && Wk && Wv && Kc && Vc && k_scale && v_scale && pos, HS2_ERR_INVALID_ARG, "null pointer");
+  HS2_CHECK(aligned16(hidden) && aligned16(Wk) && aligned16(Wv) && aligned16(Kc) && aligned16(Vc) &&
+                aligned4(k_scale) && aligned4(v_scale) && aligned4(pos),
+            HS2_ERR_INVALID_ARG, "misaligned pointer");
+  HS2_CHECK(batch >= 1 && batch <= 65535, HS2_ERR_INVALID_ARG, "batch = %d out of range", batch);
+  HS2_CHECK(hidden_dim > 0 && hidden_dim % 256 == 0, HS2_ERR_INVALID_ARG, "hidden_dim must be a positive multiple of 256");
+  HS2_CHECK(d == 256, HS2_ERR_UNSUPPORTED, "bridging supports d == 256 (got %d)", d);
+  HS2_CHECK(kv_stride_tokens >= 1, HS2_ERR_INVALID_ARG, "kv_stride_tokens must be >= 1");
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  AppendParams p;
+  p.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  p.Wk = static_cast<const __nv_bfloat16*>(Wk);
+  p.Wv = static_cast<const __nv_bfloat16*>(Wv);
+  p.kdim = hidden_dim;
+  p.Kc = static_cast<uint8_t*>(Kc);
+  p.Vc = static_cast<uint8_t*>(Vc);
+  p.ks = k_scale;
+  p.vs = v_scale;
+  p.stride = kv_stride_tokens;
+  p.pos = pos;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_begin(st);
+  bridge_append_kernel<<<dim3(BA_CLUSTER, 2, (unsigned)batch), BA_THREADS, 0, st>>>(p, ctx);
+  return after_launch("bridge_append_kernel", st);
+}
+
 hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int64_t Tq, int64_t kv_len, int Hq,
                                           int d, int window, int topk, size_t* bytes) {
   g_err[0] = 0;
@@ -496,19 +541,31 @@ hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int6
   return HS2_OK;
 }
 
-hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V, const float* k_scale,
-                                const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t q_start, int64_t Tq,
-                                int64_t kv_len, int64_t kv_stride_tokens, int Hq, int d, int window, int topk,
-                                float softmax_scale, void* O, int32_t* idx, void* workspace, size_t ws_bytes,
-                                void* stream) {
-  g_err[0] = 0;
+}  // extern "C"
+
+namespace hs2 {
+namespace {
+// hs2_full_attn_select (block == 0: topk tokens) and
+// hs2_full_attn_select_blocks (topk blocks of `block` tokens).
+hs2_status full_attn_select_impl(const void* Q, const void* K, const void* V, const float* k_scale,
+                                 const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t q_start, int64_t Tq,
+                                 int64_t kv_len, int64_t kv_stride_tokens, int Hq, int d, int window, int topk,
+                                 int block, float softmax_scale, void* O, int32_t* idx, void* workspace,
+                                 size_t ws_bytes, void* stream) {
   HS2_CHECK(Q && K && V && O && idx, HS2_ERR_INVALID_ARG, "null tensor pointer");
   HS2_CHECK(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned16(idx), HS2_ERR_INVALID_ARG,
             "tensor pointers must be 16-byte aligned");
   HS2_CHECK(batch >= 1 && Tq >= 1 && kv_len >= 1 && q_start >= 0, HS2_ERR_INVALID_ARG, "bad sizes");
   HS2_CHECK(window >= 1 && topk >= 1, HS2_ERR_INVALID_ARG, "window and topk must be >= 1");
-  HS2_CHECK(window + topk <= 2048, HS2_ERR_UNSUPPORTED, "window + topk must be <= 2048");
+  const int64_t sel_width = (int64_t)topk * (block ? block : 1);
+  HS2_CHECK(window + sel_width <= 2048, HS2_ERR_UNSUPPORTED, "the index row (window + selection) must be <= 2048");
   HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256 (got %d, %d)", Hq, d);
+  if (block) {
+    HS2_CHECK(block >= 16 && block <= 256 && (block & (block - 1)) == 0, HS2_ERR_UNSUPPORTED,
+              "block must be a power of two in [16, 256] (got %d)", block);
+    HS2_CHECK((kv_len - window + block - 1) / block <= BS_MAX_BLOCKS, HS2_ERR_UNSUPPORTED,
+              "at most %d candidate blocks per query", BS_MAX_BLOCKS);
+  }
   HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
   HS2_CHECK(kv_len - window <= (1ll << 20), HS2_ERR_UNSUPPORTED, "at most 2^20 candidate keys per query");
   HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0), HS2_ERR_WORKSPACE,
@@ -525,10 +582,10 @@ hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V, con
     HS2_CHECK(!k_scale && !v_scale, HS2_ERR_INVALID_ARG, "bf16 KV takes no scales");
     HS2_CHECK(q_start + Tq <= kv_len, HS2_ERR_INVALID_ARG, "q_start + Tq must be <= kv_len");
     HS2_CHECK(Tq * Hq < (1ll << 31) && kv_len < (1ll << 31), HS2_ERR_UNSUPPORTED, "sizes beyond int32 tiles");
-    return d == 256 ? prefill_select<256>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, softmax_scale, O, idx,
-                                          workspace, st, ctx)
-                    : prefill_select<128>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, softmax_scale, O, idx,
-                                          workspace, st, ctx);
+    return d == 256 ? prefill_select<256>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, block, softmax_scale, O,
+                                          idx, workspace, st, ctx)
+                    : prefill_select<128>(Q, K, V, q_start, Tq, kv_len, Hq, window, topk, block, softmax_scale, O,
+                                          idx, workspace, st, ctx);
   }
   HS2_CHECK(kv_dtype == HS2_KV_FP8_E4M3, HS2_ERR_INVALID_ARG, "bad kv_dtype");
   HS2_CHECK(Tq == 1 && q_start == kv_len - 1, HS2_ERR_UNSUPPORTED,
@@ -538,9 +595,34 @@ hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V, con
   HS2_CHECK(kv_stride_tokens >= kv_len, HS2_ERR_INVALID_ARG, "kv_stride_tokens must be >= kv_len");
   HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
   return d == 256 ? decode_select<256>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
-                                       softmax_scale, O, idx, workspace, st, ctx)
+                                       block, softmax_scale, O, idx, workspace, st, ctx)
                   : decode_select<128>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
-                                       softmax_scale, O, idx, workspace, st, ctx);
+                                       block, softmax_scale, O, idx, workspace, st, ctx);
+}
+}  // namespace
+}  // namespace hs2
+
+extern "C" {
+
+hs2_status hs2_full_attn_select(const void* Q, const void* K, const void* V, const float* k_scale,
+                                const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t q_start, int64_t Tq,
+                                int64_t kv_len, int64_t kv_stride_tokens, int Hq, int d, int window, int topk,
+                                float softmax_scale, void* O, int32_t* idx, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  g_err[0] = 0;
+  return full_attn_select_impl(Q, K, V, k_scale, v_scale, kv_dtype, batch, q_start, Tq, kv_len, kv_stride_tokens, Hq,
+                               d, window, topk, 0, softmax_scale, O, idx, workspace, ws_bytes, stream);
+}
+
+hs2_status hs2_full_attn_select_blocks(const void* Q, const void* K, const void* V, const float* k_scale,
+                                       const float* v_scale, hs2_kv_dtype kv_dtype, int batch, int64_t q_start,
+                                       int64_t Tq, int64_t kv_len, int64_t kv_stride_tokens, int Hq, int d, int window,
+                                       int block, int topk_blocks, float softmax_scale, void* O, int32_t* idx,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(block >= 1, HS2_ERR_INVALID_ARG, "block must be >= 1");
+  return full_attn_select_impl(Q, K, V, k_scale, v_scale, kv_dtype, batch, q_start, Tq, kv_len, kv_stride_tokens, Hq,
+                               d, window, topk_blocks, block, softmax_scale, O, idx, workspace, ws_bytes, stream);
 }
 
 hs2_status hs2_sparse_attn_prefill(const void* Q, const void* K, const void* V, const int32_t* idx, int64_t Tq,
