@@ -112,10 +112,19 @@ class ClockSampler:
 # workload arithmetic
 # ---------------------------------------------------------------------------
 
-# DRAM bytes per query row of a launch, from one ncu capture of the kernel as
-# it stands (113.3 MB read + 41.4 MB written by one T = 8192 launch); drop the
-# entry whenever the kernel changes.
-DRAM_BYTES_PER_ROW = {"sparse_tc_kernel": (113.317888e6 + 41.395456e6) / 8192}
+def dram_traffic(kernel: str):
+    """DRAM bytes per query row of one launch of `kernel`, from the ncu capture
+    recorded in profiles/dram_traffic.json, or None when there is none or when
+    the kernel's source has changed since (its SHA-256 no longer matches)."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))[kernel]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None, None
+    if hashlib.sha256(src).hexdigest() != rec["sha256"]:
+        return None, f"stale: {rec['source']} changed since the capture"
+    return rec["dram_bytes"] / rec["rows"], rec["note"]
 
 
 def prefill_flops(T, H, d, window, topk, n_sparse):
@@ -193,9 +202,20 @@ class OracleSample:
         return flops, time.perf_counter() - t0, len(rows)
 
 
-def blas_threads():
+def host_cores() -> int:
+    """Cores this process may run on (its affinity mask)."""
     try:
-        from threadpoolctl import threadpool_info
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def oracle_threads() -> int:
+    """Let the oracle's BLAS use every core of the affinity mask and return the
+    thread count it then runs with (the cores the CPU baseline actually used)."""
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+        threadpool_limits(limits=host_cores(), user_api="blas")
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return max(n) if n else 1
     except Exception:
@@ -217,6 +237,7 @@ def run_reference(args):
     w = WORKLOAD
     case = synth.make_prefill_case(w["T"], w["H"], w["d"], w["window"], w["topk"], w["n_sparse"],
                                    n_needles=w["n_needles"], scale=w["scale"], seed=0, device="cpu")
+    cores = oracle_threads()
     smp = OracleSample(case, seed=1)
     rows_per_step = args.ref_rows
     for _ in range(args.warmup):
@@ -226,13 +247,13 @@ def run_reference(args):
         f, t, n = smp.run_rows(rows_per_step)
         fl, tt, nr = fl + f, tt + t, nr + n
     value = fl / tt / 1e12
-    cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(), "sample": f"{rows_per_step} seeded rows per step"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "affinity_cores": host_cores(),
+                         "kind": "oracle",
                          "sample": f"{nr} sampled query rows of the workload (full attention + selection + "
                                    f"3 sparse layers each), {tt:.1f} s", "cpu": cpu_model()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -329,12 +350,11 @@ def run_ours(args, rank, world, dist):
     roof = None
     if dom in work:
         ach = work[dom] / (kern[dom]["avg_ms"] * 1e-3) / 1e12
-        tr = DRAM_BYTES_PER_ROW.get(dom)
+        tr, tr_note = dram_traffic(dom)
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
                 "traffic": tr * T if tr is not None else None,
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one T=8192 launch, "
-                                  "scaled by query rows (every term grows with T)" if tr is not None else None,
+                "traffic_source": tr_note,
                 "peak_source": f"{peak_src} bf16_tflops (burst: kernels of a few ms, timed one by one)"}
     sel_ms = sum(kern.get(n, {"avg_ms": 0.0})["avg_ms"] for n in ("fa_fwd_kernel", "select_sigma_kernel",
                                                                   "topk_select_kernel"))
@@ -415,9 +435,21 @@ def run_ours(args, rank, world, dist):
     # ---------------- decode over the FP8 cache
     if not args.no_decode:
         out["decode"] = bench_decode(hs2, dev, stream, flush, peaks, peak_src, args)
-    # ---------------- KV Bridging GEMM
+    # ---------------- KV Bridging GEMM, then the bridged 1M-token decode step over its caches
     if not args.no_bridge:
-        out["bridge"] = bench_bridge(hs2, dev, stream, flush, peaks, peak_src)
+        out["bridge"], bridged = bench_bridge(hs2, dev, stream, flush, peaks, peak_src)
+        if not args.no_decode:
+            out["decode_1m"] = bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged)
+        del bridged
+        torch.cuda.empty_cache()
+    # ---------------- chunked prefill at 256k and the tiny launch-bound case
+    if not args.no_long:
+        out["prefill_256k"] = bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args)
+        torch.cuda.empty_cache()
+    out["prefill_1k"] = bench_tiny(hs2, dev, stream, flush, args)
+    out["select_call_frac"] = {"prefill_32k": out["select_call"]["frac"],
+                               "prefill_256k_chunked": out.get("prefill_256k", {}).get("select_call_frac"),
+                               "peak": f"{peak_src} bf16_tflops", "target": 0.60}
 
     clocks = sampler.stop() if sampler else None
     st = hs2.hs2_device_status()
@@ -428,12 +460,14 @@ def run_ours(args, rank, world, dist):
     if rank == 0:
         out["clocks"] = clocks
         if world == 1 and not args.no_cpu:
+            cores = oracle_threads()
             smp = OracleSample(case, seed=2)
             fl, tt, nr = 0.0, 0.0, 0
             while tt < args.cpu_seconds:
                 f, t, n = smp.run_rows(16)
                 fl, tt, nr = fl + f, tt + t, nr + n
-            out["cpu_baseline"] = {"value": fl / tt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            out["cpu_baseline"] = {"value": fl / tt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                   "affinity_cores": host_cores(),
                                    "kind": "oracle", "cpu": cpu_model(),
                                    "sample": f"{nr} seeded query rows of the workload (full attention + "
                                              f"selection + 3 sparse layers per row), {tt:.1f} s"}
@@ -498,10 +532,13 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
 
 
 def bench_bridge(hs2, dev, stream, flush, peaks, peak_src):
+    """KV Bridging of 4 x 2^20 hidden rows into 2 layers' FP8 caches; returns
+    the result and the caches (the bridged decode step reads them)."""
     import synth
     c = BRIDGE
     R, D, d, L = c["R"], c["D"], c["d"], c["layers"]
     bc = synth.make_bridge_case(R, D, d, L, seed=0, device=dev)
+    bc_w = list(zip(bc.Wk, bc.Wv))
     Ks = [torch.empty(R, d, dtype=torch.uint8, device=dev) for _ in range(L)]
     Vs = [torch.empty(R, d, dtype=torch.uint8, device=dev) for _ in range(L)]
     ks = [torch.empty(R, dtype=torch.float32, device=dev) for _ in range(L)]
@@ -520,9 +557,141 @@ def bench_bridge(hs2, dev, stream, flush, peaks, peak_src):
     ms = statistics.median(t)
     flops = 2.0 * R * D * (2 * d) * L
     ach = flops / (ms * 1e-3) / 1e12
-    return {"workload": f"KV Bridging {L} layers: hidden bf16 [{R}, {D}] x W_k, W_v [{d}, {D}] -> FP8 K/V + scales",
-            "ms": ms, "achieved_tflops": ach, "peak": peaks["bf16_tflops"], "frac": ach / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16_tflops", "kernels": prof}
+    res = {"workload": f"KV Bridging {L} layers: hidden bf16 [{R}, {D}] x W_k, W_v [{d}, {D}] -> FP8 K/V + scales",
+           "ms": ms, "achieved_tflops": ach, "peak": peaks["bf16_tflops"], "frac": ach / peaks["bf16_tflops"],
+           "peak_source": f"{peak_src} bf16_tflops", "kernels": prof}
+    # the new token of each sequence (its last position), for the decode step's append
+    hid_new = bc.hidden.view(4, R // 4, D)[:, -1].contiguous()
+    del bc
+    return res, (list(zip(Ks, Vs, ks, vs)), hid_new, bc_w)
+
+
+def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged):
+    """The decode step of the 1M-token bridged workload: 4 sequences of 2^20
+    tokens, for each of the 2 cross-decoder layers (over the FP8 caches the
+    bridging GEMM just wrote) the new token's bridging + FP8 append at position
+    N - 1, full attention + selection and 3 sparse layers; L2 flushed before
+    each step."""
+    import synth
+    caches, hid_new, weights = bridged
+    c = synth.CONFIGS[5]
+    B, N, H, d, W, k, ns = c["B"], c["N"], c["H"], c["d"], c["window"], c["topk"], c["n_sparse"]
+    qs = synth.bridged_decode_queries(B, H, d, len(caches), ns, seed=0, device=dev)
+    O = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    Os = torch.empty_like(O)
+    idx = torch.empty(B, W + k, dtype=torch.int32, device=dev)
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_FP8_E4M3, B, 1, N, H, d, W, k), dev)
+    wss = hs2.workspace(hs2.hs2_sparse_attn_decode_workspace(B, W + k, H, d), dev)
+    kv = [(K.view(B, N, d), V.view(B, N, d), a.view(B, N), b.view(B, N)) for K, V, a, b in caches]
+    pos = torch.full((B,), N - 1, dtype=torch.int32, device=dev)
+
+    def step():
+        for (Kc, Vc, ksc, vsc), (Q, Qsp), (Wk, Wv) in zip(kv, qs, weights):
+            hs2.hs2_bridge_append(hid_new, Wk, Wv, Kc, Vc, ksc, vsc, pos)
+            hs2.hs2_full_attn_select(Q, Kc, Vc, O, idx, ws, window=W, topk=k, k_scale=ksc, v_scale=vsc)
+            for Qs in Qsp:
+                hs2.hs2_sparse_attn_decode(Qs, Kc, Vc, ksc, vsc, idx, Os, wss)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, args.steps)
+    hs2.hs2_profile_enable(True)
+    t = timed_steps(step, n, flush, stream)
+    prof = per_kernel(hs2.hs2_profile_collect())
+    hs2.hs2_profile_enable(False)
+    ms = statistics.median(t)
+    L = len(kv)
+    full_bytes = B * N * (2 * d + 8)
+    sp_bytes = B * ((W + k) * (2 * d + 8 + 4) + 2 * H * d * 2)
+    byte_total = L * (full_bytes + ns * sp_bytes)
+    return {"workload": f"bridged decode B={B} N={N} H={H} d={d}, {L} layers x (new-token bridging + FP8 append, "
+                        f"full + select, {ns} sparse) over the FP8 caches written by the bridging GEMM",
+            "step_ms": ms, "tok_s": B / (ms * 1e-3), "gbs": byte_total / (ms * 1e-3) / 1e9,
+            "frac": byte_total / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": byte_total,
+            "l2": "flushed before each step", "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+            "kernels": prof}
+
+
+def bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args):
+    """The long chunked prefill: T = 262144, Zipf key norms, the full layer in
+    32 query chunks of 8192 over the causal prefix, then 2 sparse layers over
+    all rows.  Inputs (2.15 GB of Q alone) are far larger than L2."""
+    import synth
+    c = synth.CONFIGS[4]
+    T, H, d, W, k, ch, ns = c["T"], c["H"], c["d"], c["window"], c["topk"], c["chunk"], c["n_sparse"]
+    if args.long_T:
+        T = args.long_T
+    case = synth.make_prefill_case(T, H, d, W, k, ns, zipf=True, scale=1.0, seed=0, device=dev)
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(T, W + k, dtype=torch.int32, device=dev)
+    Os = [torch.empty_like(O) for _ in range(ns)]
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_BF16, 1, ch, T, H, d, W, k), dev)
+
+    def step():
+        for c0 in range(0, T, ch):
+            c1 = min(T, c0 + ch)
+            hs2.hs2_full_attn_select(case.Q[c0:c1], case.K[:c1], case.V[:c1], O[c0:c1], idx[c0:c1], ws,
+                                     window=W, topk=k, q_start=c0)
+        for l in range(ns):
+            hs2.hs2_sparse_attn_prefill(case.Q_sparse[l], case.K, case.V, idx, Os[l])
+
+    step()
+    torch.cuda.synchronize()
+    hs2.hs2_profile_enable(True)
+    t = timed_steps(step, 2, lambda: None, stream)
+    prof = per_kernel(hs2.hs2_profile_collect())
+    hs2.hs2_profile_enable(False)
+    st = hs2.hs2_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {hs2.STATUS.get(st)} in the 256k prefill")
+    ms = statistics.median(t)
+    full_fl, sp1, sp_fl, sig_fl = prefill_flops(T, H, d, W, k, ns)
+    sel_ms = sum(prof.get(n, {"total_ms": 0.0})["total_ms"] for n in
+                 ("fa_fwd_kernel", "select_sigma_kernel", "topk_select_kernel")) / 2
+    sel_ach = full_fl / (sel_ms * 1e-3) / 1e12
+    sp_ms = sum(v["total_ms"] for n, v in prof.items() if "sparse" in n) / 2
+    res = {"workload": f"prefill T={T} H={H} d={d} in {ch}-query chunks over the causal prefix, Zipf key norms, "
+                       f"window {W} + top-{k}, {ns} sparse layers",
+           "step_ms": ms, "tflops": (full_fl + sp_fl) / (ms * 1e-3) / 1e12,
+           "select_call_ms": sel_ms, "select_call_tflops": sel_ach,
+           "select_call_frac": sel_ach / peaks["bf16_tflops"], "algorithmic_flops_full": full_fl,
+           "executed_extra_flops_sigma_pass": sig_fl, "sparse_ms": sp_ms,
+           "sparse_tflops": sp_fl / (sp_ms * 1e-3) / 1e12 if sp_ms > 0 else None,
+           "peak": peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16_tflops",
+           "l2": "inputs larger than L2 (Q 2.15 GB, sigma 8.6 GB per chunk)", "kernels": prof}
+    del case, O, idx, Os, ws
+    return res
+
+
+def bench_tiny(hs2, dev, stream, flush, args):
+    """The tiny single-sequence case (T = 1024, 8 heads, d = 128, window 128 +
+    top-256, 1 sparse layer): launch-bound, reported only."""
+    import synth
+    c = synth.CONFIGS[1]
+    T, H, d, W, k = c["T"], c["H"], c["d"], c["window"], c["topk"]
+    case = synth.make_prefill_case(T, H, d, W, k, c["n_sparse"], n_needles=c["n_needles"], seed=0, device=dev)
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(T, W + k, dtype=torch.int32, device=dev)
+    Os = torch.empty_like(O)
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_BF16, 1, T, T, H, d, W, k), dev)
+
+    def step():
+        hs2.hs2_full_attn_select(case.Q, case.K, case.V, O, idx, ws, window=W, topk=k)
+        hs2.hs2_sparse_attn_prefill(case.Q_sparse[0], case.K, case.V, idx, Os)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    hs2.hs2_profile_enable(True)
+    t = timed_steps(step, max(5, args.steps), flush, stream)
+    prof = per_kernel(hs2.hs2_profile_collect())
+    hs2.hs2_profile_enable(False)
+    full_fl, sp1, sp_fl, _ = prefill_flops(T, H, d, W, k, 1)
+    ms = statistics.median(t)
+    return {"workload": f"prefill T={T} H={H} d={d}, window {W} + top-{k}, 1 sparse layer, 4 needles",
+            "step_ms": ms, "tflops": (full_fl + sp_fl) / (ms * 1e-3) / 1e12,
+            "bound": "launch (4 kernels of a few microseconds each)", "kernels": prof}
 
 
 def main():
@@ -535,6 +704,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bridge", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the 256k chunked prefill")
+    ap.add_argument("--long-T", type=int, default=None, help="override the chunked prefill length (small profiling cases)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=48)
     ap.add_argument("--T", type=int, default=None, help="override the prefill length (small profiling cases)")
