@@ -212,6 +212,33 @@ def test_decode_select_fp8(hs2, B, N):
         assert max_abs(Os[b].float().numpy(), sref[b]) <= TOL_FP8
 
 
+@pytest.mark.parametrize("B,N", [(2, 140000), (1, 300000)])
+def test_decode_select_split_topk(hs2, B, N):
+    """Rows of more than 131072 candidates take the split top-k (exact top-k per
+    slice of about 32768, then one or two levels of merges of the slices'
+    lists): checked against the oracle."""
+    case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=0, seed=18)
+    O, idx = gpu_decode_select(case)
+    ref = oracle.decode_select(case.Q, case.Kc, case.Vc, case.ks, case.vs, range(B), N, 128, 1024)
+    for b in range(B):
+        ok, _, msg = check_idx_row(idx[b].numpy(), ref[b], 128, 1024)
+        assert ok, msg
+        assert max_abs(O[b].float().numpy(), ref[b].O) <= TOL_FP8
+
+
+def test_decode_split_topk_exact_ties_go_to_smaller_positions(hs2):
+    """Every key identical: every candidate score is the same fp32 value, so the
+    selection must be positions 0..1023 exactly, across the slice boundaries."""
+    B, N = 2, 300000
+    case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=0, seed=19)
+    case.Kc[:] = case.Kc[:, :1]
+    case.ks[:] = case.ks[:, :1]
+    O, idx = gpu_decode_select(case)
+    for b in range(B):
+        assert idx[b, 128:].tolist() == list(range(1024))
+        assert idx[b, :128].tolist() == list(range(N - 128, N))
+
+
 def test_sparse_decode_many_sequences(hs2):
     """More sequences than SMs' worth of splits, kv_len below the row stride."""
     B, N = 70, 3000

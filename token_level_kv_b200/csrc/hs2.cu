@@ -22,6 +22,7 @@
 #include "fa_fwd.cuh"
 #include "select_sigma.cuh"
 #include "topk.cuh"
+#include "topk_split.cuh"
 #include "sparse_tc.cuh"
 
 namespace hs2 {
@@ -197,20 +198,42 @@ PrefillWs prefill_ws(int64_t Tq, int64_t kv_len, int Hq) {
 }
 
 constexpr int kDecodeKeysPerSplit = 2048;
+
+// Slices of a decode row's top-k (topk_slice_kernel), 0 for the single-CTA
+// kernel.  The single-CTA kernel wins up to a few slices' worth of candidates
+// per row (measured: 65 us against 134 us for 64 rows of 130944); longer rows
+// are cut so that each slice and the merged lists fit one CTA's shared memory.
+int topk_split_count(int64_t n, int k) {
+  if (n <= 4 * TS_SLICE) return 0;
+  int64_t S = (n + TS_SLICE - 1) / TS_SLICE;
+  if (S * k > TS_CAP) S = TS_CAP / k;
+  if (S < 2 || S > 64) return 0;
+  if (round_up((n + S - 1) / S, 64) > TS_CAP) return 0;
+  return (int)S;
+}
+
+constexpr int kMergeGroup = 8;     // slice lists merged per CTA of the first merge level
+
 struct DecodeWs {
-  size_t logits, part, ml, sigma, total;
+  size_t logits, part, ml, sigma, lists, total;
   int64_t ld;
-  int splits;
+  int splits;        // key splits of the full-attention pass
+  int tk_splits;     // slices of the top-k (0: single CTA per row)
 };
-DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d) {
+DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d, int window, int topk) {
   DecodeWs w;
   w.ld = round_up(kv_len, 64);
   w.splits = (int)((kv_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit);
+  w.tk_splits = topk_split_count(std::max<int64_t>(0, kv_len - window), topk);
   w.logits = up256((size_t)batch * Hq * (size_t)w.ld * sizeof(float));
   w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
   w.ml = up256((size_t)batch * Hq * 2 * sizeof(float));
   w.sigma = up256((size_t)batch * (size_t)w.ld * sizeof(float));
-  w.total = w.logits + w.part + w.ml + w.sigma;
+  // slice lists, then (with more than kMergeGroup slices) the first merge level's lists
+  const int groups = w.tk_splits > kMergeGroup ? (w.tk_splits + kMergeGroup - 1) / kMergeGroup : 0;
+  w.lists = up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4)) +
+            up256((size_t)batch * groups * ((size_t)topk * 8 + 4));
+  w.total = w.logits + w.part + w.ml + w.sigma + w.lists;
   return w;
 }
 
@@ -382,7 +405,7 @@ template <int D>
 hs2_status decode_select(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
                          int64_t kv_len, int64_t kv_stride, int Hq, int window, int topk, int block, float scale,
                          void* O, int32_t* idx, void* ws, cudaStream_t st, const DevCtx& ctx) {
-  const DecodeWs w = decode_ws(batch, kv_len, Hq, D);
+  const DecodeWs w = decode_ws(batch, kv_len, Hq, D, window, topk);
   uint8_t* b = static_cast<uint8_t*>(ws);
   float* logits = reinterpret_cast<float*>(b);
   float* part = reinterpret_cast<float*>(b + w.logits);
@@ -424,6 +447,45 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
     prof_begin(st);
     decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld);
     if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
+  }
+  if (block == 0 && w.tk_splits > 0) {
+    // few rows of many candidates: the top-k split over S slices per row
+    TopkSplitParams tp;
+    uint8_t* lists = b + w.logits + w.part + w.ml + w.sigma;
+    const size_t n_list = (size_t)batch * w.tk_splits * topk;
+    tp.sigma = sigma;
+    tp.ld = w.ld;
+    tp.n = std::max<int64_t>(0, kv_len - window);
+    tp.splits = w.tk_splits;
+    tp.slice = round_up((tp.n + w.tk_splits - 1) / w.tk_splits, 64);   // 16-byte aligned slices
+    tp.topk = topk;
+    tp.window = window;
+    tp.pos = kv_len - 1;
+    tp.cval = reinterpret_cast<float*>(lists);
+    tp.cpos = reinterpret_cast<int32_t*>(lists + n_list * 4);
+    tp.ccnt = reinterpret_cast<int32_t*>(lists + n_list * 8);
+    const int groups = w.tk_splits > kMergeGroup ? (w.tk_splits + kMergeGroup - 1) / kMergeGroup : 0;
+    uint8_t* glists = lists + up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4));
+    const size_t n_glist = (size_t)batch * groups * topk;
+    tp.group = groups ? kMergeGroup : 0;
+    tp.gval = reinterpret_cast<float*>(glists);
+    tp.gpos = reinterpret_cast<int32_t*>(glists + n_glist * 4);
+    tp.gcnt = reinterpret_cast<int32_t*>(glists + n_glist * 8);
+    tp.idx = idx;
+    if ((s = set_smem(topk_slice_kernel, TS_SMEM)) != HS2_OK) return s;
+    if ((s = set_smem(topk_merge_kernel<false>, TS_SMEM)) != HS2_OK) return s;
+    if ((s = set_smem(topk_merge_kernel<true>, TS_SMEM)) != HS2_OK) return s;
+    prof_begin(st);
+    topk_slice_kernel<<<dim3((unsigned)w.tk_splits, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+    if ((s = after_launch("topk_slice_kernel", st)) != HS2_OK) return s;
+    if (groups) {
+      prof_begin(st);
+      topk_merge_kernel<false><<<dim3((unsigned)groups, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+      if ((s = after_launch("topk_merge_kernel", st)) != HS2_OK) return s;
+    }
+    prof_begin(st);
+    topk_merge_kernel<true><<<(unsigned)batch, TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+    return after_launch("topk_merge_kernel", st);
   }
   return launch_select(sigma, w.ld, kv_len - 1, 0, window, topk, block, idx, batch, st, ctx);
 }
@@ -534,7 +596,7 @@ hs2_status hs2_full_attn_select_workspace(hs2_kv_dtype kv_dtype, int batch, int6
   if (kv_dtype == HS2_KV_BF16) {
     *bytes = prefill_ws(Tq, kv_len, Hq).total;
   } else if (kv_dtype == HS2_KV_FP8_E4M3) {
-    *bytes = decode_ws(batch, kv_len, Hq, d).total;
+    *bytes = decode_ws(batch, kv_len, Hq, d, window, topk).total;
   } else {
     return fail(HS2_ERR_INVALID_ARG, "bad kv_dtype");
   }
