@@ -205,15 +205,20 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_arrive(&s_free[s]);
 
       const int64_t key0 = (int64_t)j * 128;
-      const bool diag = key0 + 127 > pq;
-      float mt = -INFINITY;
+      if (key0 + 127 > pq) {                           // the diagonal tile: keys after the query
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float v = x[i] * p.scale_log2;
-        if (diag && key0 + i > pq) v = -INFINITY;
-        x[i] = v;
-        mt = fmaxf(mt, v);
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i > pq) x[i] = -INFINITY;
       }
+      // row max of the raw scores (scale > 0 commutes with max), eight
+      // independent chains so the single warp per scheduler is not latency-bound
+      float mr[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mr[a] = x[a];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mr[i & 7] = fmaxf(mr[i & 7], x[i]);
+      const float mt = fmaxf(fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3])),
+                             fmaxf(fmaxf(mr[4], mr[5]), fmaxf(mr[6], mr[7]))) * p.scale_log2;
       const float m_new = fmaxf(m_ref, mt);
       float alpha = 1.f;
       const bool need = m_new > m_ref + 8.f;
@@ -222,12 +227,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         m_ref = m_new;
       }
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float rs = 0.f;
+      // p = 2^(s*c - mu): the argument as one packed FMA per pair, the sums in
+      // four packed accumulators
+      const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2), nmu2 = f2_pack(-mu, -mu);
+      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        x[i] = fast_exp2(x[i] - mu);
-        rs += x[i];
+      for (int i = 0; i < 128; i += 2) {
+        const float2 a = f2_unpack(ffma2(f2_pack(x[i], x[i + 1]), c2, nmu2));
+        x[i] = fast_exp2(a.x);
+        x[i + 1] = fast_exp2(a.y);
+        rs2[(i >> 1) & 3] = fadd2(rs2[(i >> 1) & 3], f2_pack(x[i], x[i + 1]));
       }
+      const float2 r01 = f2_unpack(fadd2(rs2[0], rs2[1])), r23 = f2_unpack(fadd2(rs2[2], rs2[3]));
+      const float rs = (r01.x + r01.y) + (r23.x + r23.y);
       l = l * alpha + rs;
 
       if (j >= 1) {

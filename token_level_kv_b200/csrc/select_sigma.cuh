@@ -57,7 +57,7 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* ring = smem + L::OFF_RING;
-  float* sML = reinterpret_cast<float*>(smem + L::OFF_ML);     // [256][2]: m, 1/l
+  float* sML = reinterpret_cast<float*>(smem + L::OFF_ML);     // [256] -m, then [256] 1/l
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* full = bars + 1;                    // [SG_STAGES]
@@ -96,8 +96,8 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
       const float l = p.ml[R * 2 + 1];
       inv = l > 0.f ? 1.f / l : 0.f;
     }
-    sML[i * 2] = m;
-    sML[i * 2 + 1] = inv;
+    sML[i] = -m;
+    sML[256 + i] = inv;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -188,18 +188,27 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
 #pragma unroll
         for (int c = 0; c < 2; ++c) tmem_ld16(lane_base + buf * 256 + part * 64 + c0 + c * 16, v + c * 16);
         tmem_wait_ld();
-        // column part*64 + c0 + i  <->  (query (part*64 + c0 + i) / H, head i % H)
+        // column part*64 + c0 + i  <->  (query (part*64 + c0 + i) / H, head i % H);
+        // heads in pairs: one packed FMA for the two exponents' arguments and
+        // one for the two terms of the sum (two interleaved partial sums)
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
         for (int qi = 0; qi < 32 / H; ++qi) {
           const int col = part * 64 + c0 + qi * H;
           const int64_t tq = g0 + col / H;
           const int64_t pq = p.q_start + tq;
-          const float* ml = sML + (size_t)col * 2;
-          float acc = 0.f;
+          uint64_t acc2 = 0ull;
 #pragma unroll
-          for (int h = 0; h < H; ++h)
-            acc += fast_exp2(fmaf(v[qi * H + h], p.scale_log2, -ml[2 * h])) * ml[2 * h + 1];
-          if (tq < p.Tq && key <= pq - p.window) p.sigma[tq * p.ld + key] = acc;
+          for (int h = 0; h < H; h += 4) {
+            const float4 nm = *reinterpret_cast<const float4*>(sML + col + h);        // -m of 4 heads
+            const float4 iv = *reinterpret_cast<const float4*>(sML + 256 + col + h);  // 1/l of 4 heads
+            const float2 a = f2_unpack(ffma2(f2_pack(v[qi * H + h], v[qi * H + h + 1]), c2, f2_pack(nm.x, nm.y)));
+            const float2 b = f2_unpack(ffma2(f2_pack(v[qi * H + h + 2], v[qi * H + h + 3]), c2, f2_pack(nm.z, nm.w)));
+            acc2 = ffma2(f2_pack(fast_exp2(a.x), fast_exp2(a.y)), f2_pack(iv.x, iv.y), acc2);
+            acc2 = ffma2(f2_pack(fast_exp2(b.x), fast_exp2(b.y)), f2_pack(iv.z, iv.w), acc2);
+          }
+          const float2 r = f2_unpack(acc2);
+          if (tq < p.Tq && key <= pq - p.window) p.sigma[tq * p.ld + key] = r.x + r.y;
         }
       }
       tc_fence_before();
