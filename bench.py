@@ -163,6 +163,26 @@ def timed_steps(step, steps, flush, stream):
     return [a.elapsed_time(b) for a, b in ts]
 
 
+def graph_step_ms(step, n, flush, stream):
+    """The step captured once as a CUDA graph and replayed (L2 flushed before
+    each replay): the launch gaps between its kernels go away."""
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()                                   # warm on the capture stream
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(timed_steps(g.replay, n, flush, stream))
+    del g
+    return ms
+
+
 def per_kernel(records):
     agg = {}
     for name, ms in records:
@@ -504,6 +524,12 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
     prof_sp = per_kernel(hs2.hs2_profile_collect())
     hs2.hs2_profile_enable(False)
     t_warm = timed_steps(lambda: [sparse(l) for l in range(c["n_sparse"])], n, lambda: None, stream)
+
+    def whole_step():
+        full()
+        for l in range(c["n_sparse"]):
+            sparse(l)
+    g_ms = graph_step_ms(whole_step, n, flush, stream)
     prof = {"full_select_call": prof_full, "sparse_call": prof_sp}
     ms_full = statistics.median(t_full)
     ms_sp = [statistics.median(t) for t in t_sp]
@@ -518,6 +544,7 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
         "workload": f"decode B={B} N={N} H={H} d={d} FP8 E4M3 cache + per-token scales, "
                     f"window {W} + top-{k}, 3 sparse layers",
         "tok_s": B / (step_ms * 1e-3), "step_ms": step_ms,
+        "step_ms_cuda_graph": g_ms, "tok_s_cuda_graph": B / (g_ms * 1e-3),
         "full_select_ms": ms_full, "full_select_gbs": full_gbs, "full_select_frac": full_gbs / peaks["hbm_gbs"],
         "sparse_ms": ms_sp, "sparse_gbs": sp_gbs, "sparse_frac": sp_gbs / peaks["hbm_gbs"],
         "sparse_kernel_ms": sp_kernel_ms,
@@ -601,6 +628,7 @@ def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged
     prof = per_kernel(hs2.hs2_profile_collect())
     hs2.hs2_profile_enable(False)
     ms = statistics.median(t)
+    g_ms = graph_step_ms(step, n, flush, stream)
     L = len(kv)
     full_bytes = B * N * (2 * d + 8)
     sp_bytes = B * ((W + k) * (2 * d + 8 + 4) + 2 * H * d * 2)
@@ -608,6 +636,7 @@ def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged
     return {"workload": f"bridged decode B={B} N={N} H={H} d={d}, {L} layers x (new-token bridging + FP8 append, "
                         f"full + select, {ns} sparse) over the FP8 caches written by the bridging GEMM",
             "step_ms": ms, "tok_s": B / (ms * 1e-3), "gbs": byte_total / (ms * 1e-3) / 1e9,
+            "step_ms_cuda_graph": g_ms, "tok_s_cuda_graph": B / (g_ms * 1e-3),
             "frac": byte_total / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": byte_total,
             "l2": "flushed before each step", "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
             "kernels": prof}
