@@ -64,20 +64,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_amn(int M, int N) {
   return umma_idesc_bf16(M, N, false) | (1u << 15);
 }
 
-// Barrier `id` over `n` threads that also ANDs a predicate across them.
-__device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred q, s;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "barrier.cta.red.and.pred s, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, s;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
 template <int D>
 __global__ void __launch_bounds__(StcLayout<D>::NT, 1)
 sparse_tc_kernel(Attn16Params p, DevCtx ctx) {

@@ -315,7 +315,11 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
   uint32_t lo, hi, krem, in_range;
   // With win_hi < 0x7f800000 the first pass bins only [win_lo, win_hi] (every
   // candidate is >= win_lo) plus one overflow bin for the candidates above.
-  auto range_select = [&](uint32_t r, uint32_t count, uint32_t win_lo, uint32_t win_hi) {
+  // With coarse > 0 the select stops as soon as the bin holding the r-th
+  // element holds at most `coarse` elements: lo is then a pattern with between
+  // r and r + coarse - 1 listed elements at or above it (a bound, not the
+  // exact r-th pattern).
+  auto range_select = [&](uint32_t r, uint32_t count, uint32_t win_lo, uint32_t win_hi, uint32_t coarse) {
     lo = win_lo;
     hi = win_hi;
     krem = r;
@@ -359,6 +363,7 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
         hi = (top > hi || top < nlo) ? hi : top;
       }
       over = false;
+      if (coarse && in_range <= coarse) break;
       if (!listed && r - krem + in_range <= (uint32_t)TK_CAP) {
         collect(lo);                         // exactly r - krem + in_range of them
         listed = true;
@@ -410,23 +415,25 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
     __syncthreads();
     listed = true;
     if (sb == 1) {
-      range_select(k, (uint32_t)n, 0u, 0x7f800000u);   // the whole row is the sample
+      range_select(k, (uint32_t)n, 0u, 0x7f800000u, 0u);   // the whole row is the sample
     } else {
       const float ks = (float)k * (float)m / (float)n;
       const uint32_t rv = min(m, (uint32_t)(ks + 4.f * sqrtf(ks) + 8.f));
       // the row into L2 while the sample is searched (the next pass reads it all)
       for (int64_t i = (int64_t)threadIdx.x * 32; i < n; i += 32 * TK_THREADS)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i));
-      range_select(rv, m, 0u, 0x7f800000u);
+      // the bound needs only the bin of the rv-th sample pattern, not the
+      // pattern itself: one pass unless that bin is crowded
+      range_select(rv, m, 0u, 0x7f800000u, 16u);
       const uint32_t V = lo;
       collect(V);
       if (ncand >= k && ncand <= (uint32_t)TK_CAP) {
         // T is within a few sample ranks of V: first look 2^16 patterns above it
-        if (V < 0x7f7f0000u) range_select(k, ncand, V, V + 0xffffu);
-        else range_select(k, ncand, 0u, 0x7f800000u);
+        if (V < 0x7f7f0000u) range_select(k, ncand, V, V + 0xffffu, 0u);
+        else range_select(k, ncand, 0u, 0x7f800000u, 0u);
       } else {
         listed = false;
-        range_select(k, (uint32_t)n, 0u, 0x7f800000u);
+        range_select(k, (uint32_t)n, 0u, 0x7f800000u, 0u);
       }
     }
   }
