@@ -279,6 +279,62 @@ def sparse_attn(Qs: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Self-decoder sliding-window attention with partial RoPE
+# ---------------------------------------------------------------------------
+
+def rope_rows(X: np.ndarray, positions: np.ndarray, rope_dims: int = 64,
+              base: float = 10000.0) -> np.ndarray:
+    """Rotary position embedding on the first rope_dims dims of every row
+    (agihunt.info summary: the SWA layers use 64-dim partial RoPE; full and
+    sparse layers use NoPE).  Readings, the pages fixing none of them: pairs
+    are (i, i + rope_dims/2) for i < rope_dims/2 (rotate-half), the angle of
+    pair i at position p is p * base^(-2i/rope_dims) with base 10000, and the
+    remaining dims pass through.
+
+    X: [..., rows, d] (any leading dims), positions: [rows] absolute positions.
+    """
+    X = f64(X)
+    half = rope_dims // 2
+    inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / rope_dims)   # [half]
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]    # [rows, half]
+    shape = [1] * (X.ndim - 2) + [ang.shape[0], half]
+    c = np.cos(ang).reshape(shape)
+    sn = np.sin(ang).reshape(shape)
+    out = X.copy()
+    x1 = X[..., :half]
+    x2 = X[..., half:rope_dims]
+    out[..., :half] = x1 * c - x2 * sn
+    out[..., half:rope_dims] = x1 * sn + x2 * c
+    return out
+
+
+def swa_attn(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rows: Sequence[int], q_start: int,
+             window: int, rope_dims: int = 64, base: float = 10000.0,
+             scale: Optional[float] = None) -> Dict[int, np.ndarray]:
+    """Sliding-window causal attention of the self-decoder (agihunt.info summary,
+    backbone paragraph: each query attends only to the most recent tokens), MQA
+    with one KV head, RoPE on q and k: query t at position p = q_start + t sees
+    keys [max(0, p - window + 1), p].
+
+    Q: [Tq, H, d]; K, V: [kv_len, d].  Returns {t: O [H, d]} (unrounded).
+    """
+    d = Q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    Kr = rope_rows(K, np.arange(K.shape[0]), rope_dims, base)
+    V = f64(V)
+    out = {}
+    for t in rows:
+        p = q_start + t
+        q = rope_rows(f64(Q[t])[None], np.array([p]), rope_dims, base)[0]   # [H, d]
+        lo = max(0, p - window + 1)
+        s = (q @ Kr[lo:p + 1].T) * scale
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        out[t] = (e / e.sum(axis=1, keepdims=True)) @ V[lo:p + 1]
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Decode over the FP8 cache
 # ---------------------------------------------------------------------------
 

@@ -484,3 +484,72 @@ def test_block_selection_uniform_closed_form():
         nb = b.block_score.shape[0]
         expect = list(range(min(k, nb))) if full >= k or nb <= k else list(range(full)) + [nb - 1]
         assert b.blocks.tolist() == expect
+
+
+# ---------------------------------------------------------------- SWA with partial RoPE
+
+def test_rope_preserves_pair_norms_and_leaves_the_rest():
+    X = _rand((7, 3, 96), 900)
+    pos = np.array([0, 1, 5, 77, 1000, 65535, 262143])
+    Y = oracle.rope_rows(X.transpose(1, 0, 2), pos).transpose(1, 0, 2)     # rows on axis -2
+    assert np.array_equal(Y[..., 64:], X[..., 64:])                        # dims past 64 untouched
+    n_x = X[..., :32] ** 2 + X[..., 32:64] ** 2
+    n_y = Y[..., :32] ** 2 + Y[..., 32:64] ** 2
+    assert np.allclose(n_y, n_x, rtol=1e-12)
+    assert np.allclose(Y[0], X[0], rtol=0, atol=0)                          # position 0: identity
+
+
+def test_rope_scores_depend_only_on_the_distance():
+    """<rope(q, m), rope(k, n)> is a function of m - n: shifting both positions
+    by the same amount leaves every score unchanged, and the score at distance
+    0 is the plain dot product on the rotated dims."""
+    q = _rand((1, 64), 901)
+    k = _rand((1, 64), 902)
+    for m, n in ((10, 3), (5000, 4993), (123456, 123449)):
+        a = oracle.rope_rows(q, np.array([m])) @ oracle.rope_rows(k, np.array([n])).T
+        b = oracle.rope_rows(q, np.array([m - n])) @ oracle.rope_rows(k, np.array([0])).T
+        assert np.allclose(a, b, rtol=1e-9, atol=1e-9)
+    same = oracle.rope_rows(q, np.array([777])) @ oracle.rope_rows(k, np.array([777])).T
+    assert np.allclose(same, q @ k.T, rtol=1e-10)
+    # a planted mistake: pairs (2i, 2i+1) instead of (i, i + 32) keep norms but
+    # break the distance rule against this pairing's rotation of the same vector
+    def rope_interleaved(x, p):
+        inv = 10000.0 ** (-2.0 * np.arange(32) / 64)
+        ang = p * inv
+        y = x.copy()
+        y[:, 0:64:2] = x[:, 0:64:2] * np.cos(ang) - x[:, 1:64:2] * np.sin(ang)
+        y[:, 1:64:2] = x[:, 0:64:2] * np.sin(ang) + x[:, 1:64:2] * np.cos(ang)
+        return y
+    assert not np.allclose(rope_interleaved(q, 10), oracle.rope_rows(q, np.array([10])))
+
+
+@pytest.mark.parametrize("T,W,q_start", [(70, 16, 0), (40, 8, 25), (33, 100, 0)])
+def test_swa_matches_sdpa_with_a_band_mask(T, W, q_start):
+    H, d = 3, 80
+    kv = q_start + T
+    q = _rand((T, H, d), 903)
+    K = _rand((kv, d), 904)
+    V = _rand((kv, d), 905)
+    got = oracle.swa_attn(q, K, V, range(T), q_start, W)
+    # torch: rotate with the oracle's RoPE (pinned above), then fp64 SDPA with
+    # the band mask of the window
+    qr = np.stack([oracle.rope_rows(q[t][None], np.array([q_start + t]))[0] for t in range(T)])
+    kr = oracle.rope_rows(K, np.arange(kv))
+    pos = q_start + np.arange(T)[:, None]
+    key = np.arange(kv)[None, :]
+    mask = (key <= pos) & (key > pos - W)
+    ref = _sdpa(qr, kr, V, mask=mask)
+    for t in range(T):
+        assert np.allclose(got[t], ref[t], rtol=1e-12, atol=1e-12)
+
+
+def test_swa_with_a_window_over_the_prefix_is_causal_attention():
+    """A window at least as long as the prefix is plain causal attention over the
+    rotated q and k: the same as the full-attention oracle on rotated inputs."""
+    T, H, d = 50, 4, 64
+    q, K, V = _rand((T, H, d), 906), _rand((T, d), 907), _rand((T, d), 908)
+    got = oracle.swa_attn(q, K, V, range(T), 0, window=T)
+    qr = np.stack([oracle.rope_rows(q[t][None], np.array([t]))[0] for t in range(T)])
+    full = oracle.full_attn_select(qr, oracle.rope_rows(K, np.arange(T)), V, range(T), 0, 4, 3)
+    for t in range(T):
+        assert np.allclose(got[t], full[t].O, rtol=1e-12, atol=1e-12)
