@@ -246,6 +246,34 @@ HS2_API hs2_status hs2_sparse_attn_decode_static(const void* Q, const void* Kc, 
                                          void* stream);
 
 /*
+ * Sliding-window attention of a self-decoder SWA layer, with partial RoPE
+ * (agihunt.info summary: the self-decoder mixes full and sliding-window
+ * attention, each SWA query attending only to the most recent tokens; SWA
+ * layers use 64-dim partial RoPE, the full and sparse layers NoPE; MQA).
+ * These layers produce the hidden states the KV Bridging consumes.  Query t
+ * sits at absolute position p = q_start + t and attends to keys
+ * [max(0, p - window + 1), p]:
+ *     O[t,h,:] = sum_j softmax_j(scale * rope(q_th, p) . rope(k_j, j)) v_j
+ * rope(x, p) rotates the pairs (x_i, x_{i+R/2}), i < R/2 = rope_dims/2, by the
+ * angle p * rope_base^(-2i/R) and leaves the dims from R on unchanged.  The
+ * rotated q and k are rounded to bf16 before the products (fp32 accumulation).
+ *   Q bf16 [Tq, Hq, d]; K, V bf16 [kv_len, d] (one KV head); O bf16 [Tq, Hq, d].
+ *   workspace: at least hs2_swa_attn_prefill_workspace() bytes, 256-byte
+ *   aligned (the rotated Q and K and a cos/sin table); contents on entry do
+ *   not matter.
+ * Requires q_start + Tq <= kv_len, window >= 1, rope_dims in {16, 32, 64},
+ * rope_base > 1 (10000 is the usual value), and the shapes of
+ * hs2_full_attn_select's prefill.
+ */
+HS2_API hs2_status hs2_swa_attn_prefill(const void* Q, const void* K, const void* V, int64_t q_start,
+                                        int64_t Tq, int64_t kv_len, int Hq, int d, int window,
+                                        int rope_dims, float rope_base, float softmax_scale, void* O,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
+HS2_API hs2_status hs2_swa_attn_prefill_workspace(int64_t Tq, int64_t kv_len, int Hq, int d,
+                                                  int rope_dims, size_t* bytes);
+
+/*
  * Synchronises `stream`, then reads and clears the status word of the current
  * device: HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA if
  * the synchronisation itself failed).

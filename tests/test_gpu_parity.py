@@ -194,6 +194,39 @@ def test_decode_block_selection_fp8(hs2):
         assert max_abs(O[b].float().cpu().numpy(), ref[b].O) <= TOL_FP8
 
 
+@pytest.mark.parametrize("T,H,d,W,q_start", [(1500, 16, 256, 128, 0), (1500, 8, 128, 64, 0), (900, 16, 256, 300, 700),
+                                            (100, 16, 256, 128, 0), (2600, 16, 128, 1, 0)])
+def test_swa_attn_partial_rope(hs2, T, H, d, W, q_start):
+    """Self-decoder sliding-window attention with 64-dim partial RoPE against
+    the oracle: windows of 1, 64, 128 and 300 keys, a query block starting at
+    700 over the causal prefix, rows with fewer keys than the window."""
+    kv = q_start + T
+    case = synth.make_prefill_case(kv, H, d, W, 8, n_sparse=0, seed=20)
+    Q = case.Q[q_start:kv].cuda().contiguous()
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device="cuda")
+    ws = hs2.workspace(hs2.hs2_swa_attn_prefill_workspace(T, kv, H, d))
+    hs2.hs2_swa_attn_prefill(Q, case.K.cuda(), case.V.cuda(), O, ws, window=W, q_start=q_start)
+    assert hs2.hs2_device_status() == 0
+    rows = sorted(set(list(range(0, T, 29)) + [0, 1, W - 1, W, W + 1, T - 1]) & set(range(T)))
+    ref = oracle.swa_attn(case.Q[q_start:kv], case.K, case.V, rows, q_start, W)
+    Oc = O.float().cpu().numpy()
+    assert max(max_abs(Oc[t], ref[t]) for t in rows) <= TOL_BF16
+
+
+def test_swa_chunked_equals_one_call(hs2):
+    T, H, d, W = 1800, 16, 256, 128
+    case = synth.make_prefill_case(T, H, d, W, 8, n_sparse=0, seed=21)
+    Q, K, V = case.Q.cuda(), case.K.cuda(), case.V.cuda()
+    ws = hs2.workspace(hs2.hs2_swa_attn_prefill_workspace(T, T, H, d))
+    O1 = torch.empty(T, H, d, dtype=torch.bfloat16, device="cuda")
+    hs2.hs2_swa_attn_prefill(Q, K, V, O1, ws, window=W)
+    O2 = torch.empty_like(O1)
+    hs2.hs2_swa_attn_prefill(Q[:904].contiguous(), K, V, O2[:904], ws, window=W, kv_len=904)
+    hs2.hs2_swa_attn_prefill(Q[904:].contiguous(), K, V, O2[904:], ws, window=W, q_start=904)
+    assert hs2.hs2_device_status() == 0
+    assert torch.equal(O1, O2)
+
+
 # ---------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("B,N", [(3, 5000), (2, 1200), (1, 100), (2, 4097)])

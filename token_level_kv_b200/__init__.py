@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
         "hs2_sparse_attn_decode": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P, Z, P], I),
         "hs2_sparse_attn_decode_workspace": ([I, I, I, I, ctypes.POINTER(Z)], I),
         "hs2_sparse_attn_decode_static": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P], I),
+        "hs2_swa_attn_prefill": ([P, P, P, L, L, L, I, I, I, I, F, F, P, P, Z, P], I),
+        "hs2_swa_attn_prefill_workspace": ([L, L, I, I, I, ctypes.POINTER(Z)], I),
         "hs2_device_status": ([P], I),
         "hs2_set_spin_limit": ([L], I),
         "hs2_profile_enable": ([I], I),
@@ -67,7 +69,7 @@ EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv"
            "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
            "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit",
            "hs2_profile_enable", "hs2_profile_collect", "hs2_sparse_attn_decode_static", "hs2_bridge_append",
-           "hs2_full_attn_select_blocks")
+           "hs2_full_attn_select_blocks", "hs2_swa_attn_prefill", "hs2_swa_attn_prefill_workspace")
 
 
 def _check(status: int) -> None:
@@ -176,6 +178,25 @@ def _select_args(Q, K, q_start, kv_len, softmax_scale, workspace) -> dict:
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return dict(kvd=kvd, d=d, H=H, scale=scale, batch=batch, Tq=Tq, kv_len=kv_len, stride=stride, q_start=q_start,
                 ws=ws)
+
+
+def hs2_swa_attn_prefill_workspace(Tq: int, kv_len: int, Hq: int, d: int, rope_dims: int = 64) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hs2_swa_attn_prefill_workspace(Tq, kv_len, Hq, d, rope_dims, ctypes.byref(n)))
+    return n.value
+
+
+def hs2_swa_attn_prefill(Q, K, V, O, workspace, *, window: int, q_start: int = 0, kv_len: int | None = None,
+                         rope_dims: int = 64, rope_base: float = 10000.0, softmax_scale: float | None = None,
+                         stream=None) -> None:
+    """Sliding-window attention with partial RoPE: Q [Tq, H, d] at positions
+    q_start.. over K, V [>= kv_len, d]; O [Tq, H, d]."""
+    Tq, H, d = Q.shape
+    kv_len = K.shape[0] if kv_len is None else kv_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.hs2_swa_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), q_start, Tq, kv_len, H, d, window, rope_dims,
+                                    rope_base, scale, _ptr(O), _ptr(workspace), ws, _stream(stream)))
 
 
 def hs2_sparse_attn_prefill(Q, K, V, idx, O, *, kv_len: int | None = None, softmax_scale: float | None = None,

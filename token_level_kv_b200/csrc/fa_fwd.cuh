@@ -46,8 +46,9 @@ struct FaParams {
   int H;
   float scale_log2;        // softmax_scale * log2(e)
   __nv_bfloat16* O;        // [Tq*H, D]
-  float* ml;               // [Tq*H, 2]: m (log2 units, the reference max used), l
+  float* ml;               // [Tq*H, 2]: m (log2 units, the reference max used), l; may be null
   int n_qtiles;
+  int64_t window;          // 0: every key <= the query; else the keys [p - window + 1, p]
 };
 
 template <int D>
@@ -81,7 +82,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int64_t q0 = (int64_t)qt * qpt;
   const int64_t q_last = min(p.Tq, q0 + qpt) - 1;
   const int64_t p_last = p.q_start + q_last;
-  const int n_kt = (int)(p_last / 128) + 1;
+  // key tiles kt0 .. kt0 + n_kt - 1 (a sliding window starts at the first
+  // query's oldest key); loop counters j run from 0 and the tile is kt0 + j
+  const int kt0 = p.window > 0 ? (int)(max((int64_t)0, p.q_start + q0 - p.window + 1) / 128) : 0;
+  const int n_kt = (int)(p_last / 128) + 1 - kt0;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -119,7 +123,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int j = 0; j < n_kt; ++j) {
         if (!mbar_wait(k_empty, (j & 1) ^ 1, ctx)) break;
         mbar_expect_tx(k_full, L::K_BYTES);
-        for (int b = 0; b < D / 64; ++b) tma_load_2d(sK + b * 16384, &tmK, k_full, b * 64, j * 128);
+        for (int b = 0; b < D / 64; ++b) tma_load_2d(sK + b * 16384, &tmK, k_full, b * 64, (kt0 + j) * 128);
         last = j;
       }
       mbar_drain(q_full, 0);
@@ -133,7 +137,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int j = 0; j < n_kt; ++j) {
         if (!mbar_wait(v_empty, (j & 1) ^ 1, ctx)) break;
         mbar_expect_tx(v_full, L::V_BYTES);
-        for (int b = 0; b < D / 64; ++b) tma_load_2d(sV + b * 16384, &tmV, v_full, b * 64, j * 128);
+        for (int b = 0; b < D / 64; ++b) tma_load_2d(sV + b * 16384, &tmV, v_full, b * 64, (kt0 + j) * 128);
         last = j;
       }
       if (last >= 0) mbar_drain(v_full, last & 1);
@@ -204,11 +208,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_before();
       mbar_arrive(&s_free[s]);
 
-      const int64_t key0 = (int64_t)j * 128;
+      const int64_t key0 = (int64_t)(kt0 + j) * 128;
       if (key0 + 127 > pq) {                           // the diagonal tile: keys after the query
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (key0 + i > pq) x[i] = -INFINITY;
+      }
+      if (p.window > 0 && key0 <= pq - p.window) {     // keys older than the sliding window
+        const int64_t oldest = pq - p.window + 1;
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i < oldest) x[i] = -INFINITY;
       }
       // row max of the raw scores (scale > 0 commutes with max), eight
       // independent chains so the single warp per scheduler is not latency-bound
@@ -291,7 +301,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (valid) {
+      if (valid && p.ml) {
         p.ml[R * 2] = m_ref;
         p.ml[R * 2 + 1] = l;
       }

@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "decode_attn.cuh"
 #include "fa_fwd.cuh"
+#include "rope_swa.cuh"
 #include "select_sigma.cuh"
 #include "topk.cuh"
 #include "topk_split.cuh"
@@ -174,10 +175,38 @@ hs2_status after_launch(const char* what, cudaStream_t st) {
   return HS2_OK;
 }
 
+// Raises a kernel's dynamic shared memory limit on the current device, once
+// per (kernel, device, size): the attribute call costs microseconds of host
+// time, which small decode launches would otherwise pay every call.
+struct SmemSet {
+  const void* kernel;
+  int dev;
+  size_t bytes;
+};
+constexpr int kMaxSmemSet = 256;
+SmemSet g_smem_set[kMaxSmemSet];
+int g_n_smem_set = 0;
+
 template <typename K>
 hs2_status set_smem(K kernel, size_t bytes) {
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const void* kp = reinterpret_cast<const void*>(kernel);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_n_smem_set; ++i)
+      if (g_smem_set[i].kernel == kp && g_smem_set[i].dev == dev && g_smem_set[i].bytes >= bytes) return HS2_OK;
+  }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_n_smem_set; ++i)
+    if (g_smem_set[i].kernel == kp && g_smem_set[i].dev == dev) {
+      if (bytes > g_smem_set[i].bytes) g_smem_set[i].bytes = bytes;
+      return HS2_OK;
+    }
+  if (g_n_smem_set < kMaxSmemSet) g_smem_set[g_n_smem_set++] = {kp, dev, bytes};
   return HS2_OK;
 }
 
@@ -341,10 +370,13 @@ hs2_status launch_select(const float* sigma, int64_t ld, int64_t p0, int64_t pst
   bp.window = window;
   bp.block = block;
   bp.topk_blocks = topk;
+  // the last row has the most candidates (prefill: the largest position; decode: all rows alike)
+  bp.nb_max = (int)((std::max<int64_t>(0, p0 + (rows - 1) * pstep - window + 1) + block - 1) / block);
   bp.idx = idx;
-  if ((s = set_smem(block_select_kernel, BS_SMEM)) != HS2_OK) return s;
+  const size_t smem = bs_smem(bp.nb_max);
+  if ((s = set_smem(block_select_kernel, smem)) != HS2_OK) return s;
   prof_begin(st);
-  block_select_kernel<<<(unsigned)rows, BS_THREADS, BS_SMEM, st>>>(bp, ctx);
+  block_select_kernel<<<(unsigned)rows, BS_THREADS, smem, st>>>(bp, ctx);
   return after_launch("block_select_kernel", st);
 }
 
@@ -372,6 +404,7 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
   fp.O = static_cast<__nv_bfloat16*>(O);
   fp.ml = ml;
   fp.n_qtiles = (int)((Tq * Hq + 127) / 128);
+  fp.window = 0;
   if ((s = set_smem(fa_fwd_kernel<D>, FaLayout<D>::SMEM)) != HS2_OK) return s;
   prof_begin(st);
   fa_fwd_kernel<D><<<fp.n_qtiles, FA_THREADS, FaLayout<D>::SMEM, st>>>(mQ, mK, mV, fp, ctx);
@@ -488,6 +521,62 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
     return after_launch("topk_merge_kernel", st);
   }
   return launch_select(sigma, w.ld, kv_len - 1, 0, window, topk, block, idx, batch, st, ctx);
+}
+
+struct SwaWs {
+  size_t q, k, table, total;
+};
+SwaWs swa_ws(int64_t Tq, int64_t kv_len, int Hq, int d, int rope_dims) {
+  SwaWs w;
+  w.q = up256((size_t)Tq * Hq * d * 2);
+  w.k = up256((size_t)kv_len * d * 2);
+  w.table = up256((size_t)kv_len * (rope_dims / 2) * sizeof(float2));
+  w.total = w.q + w.k + w.table;
+  return w;
+}
+
+// Sliding-window attention of the self-decoder: RoPE on Q and K into the
+// workspace, then the full-attention kernel over each query's window.
+template <int D>
+hs2_status swa_attn(const void* Q, const void* K, const void* V, int64_t q_start, int64_t Tq, int64_t kv_len, int Hq,
+                    int window, int rope_dims, float rope_base, float scale, void* O, void* ws, cudaStream_t st,
+                    const DevCtx& ctx) {
+  const SwaWs w = swa_ws(Tq, kv_len, Hq, D, rope_dims);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* Qr = reinterpret_cast<__nv_bfloat16*>(b);
+  __nv_bfloat16* Kr = reinterpret_cast<__nv_bfloat16*>(b + w.q);
+  float2* cs = reinterpret_cast<float2*>(b + w.q + w.k);
+  const int half = rope_dims / 2;
+  hs2_status s;
+  prof_begin(st);
+  rope_table_kernel<<<(unsigned)((kv_len * half + 255) / 256), 256, 0, st>>>(cs, kv_len, half, (double)rope_base);
+  if ((s = after_launch("rope_table_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  rope_rows_kernel<D><<<(unsigned)((Tq * Hq + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), Qr,
+                                                                      Tq * Hq, q_start, Hq, cs, half);
+  if ((s = after_launch("rope_rows_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  rope_rows_kernel<D><<<(unsigned)((kv_len + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(K), Kr, kv_len,
+                                                                     0, 1, cs, half);
+  if ((s = after_launch("rope_rows_kernel", st)) != HS2_OK) return s;
+  CUtensorMap mQ, mK, mV;
+  if ((s = make_map_bf16(&mQ, Qr, D, (uint64_t)Tq * Hq, D, 64, 128)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mK, Kr, D, (uint64_t)kv_len, D, 64, 128)) != HS2_OK) return s;
+  if ((s = make_map_bf16(&mV, V, D, (uint64_t)kv_len, D, 64, 128)) != HS2_OK) return s;
+  FaParams fp;
+  fp.Tq = Tq;
+  fp.q_start = q_start;
+  fp.kv_len = kv_len;
+  fp.H = Hq;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  fp.O = static_cast<__nv_bfloat16*>(O);
+  fp.ml = nullptr;
+  fp.n_qtiles = (int)((Tq * Hq + 127) / 128);
+  fp.window = window;
+  if ((s = set_smem(fa_fwd_kernel<D>, FaLayout<D>::SMEM)) != HS2_OK) return s;
+  prof_begin(st);
+  fa_fwd_kernel<D><<<fp.n_qtiles, FA_THREADS, FaLayout<D>::SMEM, st>>>(mQ, mK, mV, fp, ctx);
+  return after_launch("fa_fwd_kernel", st);
 }
 
 }  // namespace
@@ -848,6 +937,44 @@ hs2_status hs2_sparse_attn_decode_static(const void* Q, const void* Kc, const vo
   if ((s = static_scratch_ptr(&scratch)) != HS2_OK) return s;
   return hs2_sparse_attn_decode(Q, Kc, Vc, k_scale, v_scale, kv_dtype, batch, kv_len, kv_stride_tokens, idx,
                                 n_idx, Hq, d, softmax_scale, O, scratch, HS2_STATIC_SCRATCH_BYTES, stream);
+}
+
+hs2_status hs2_swa_attn_prefill_workspace(int64_t Tq, int64_t kv_len, int Hq, int d, int rope_dims, size_t* bytes) {
+  g_err[0] = 0;
+  HS2_CHECK(bytes, HS2_ERR_INVALID_ARG, "bytes is null");
+  HS2_CHECK(Tq >= 1 && kv_len >= 1, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  HS2_CHECK(rope_dims == 16 || rope_dims == 32 || rope_dims == 64, HS2_ERR_UNSUPPORTED,
+            "rope_dims must be 16, 32 or 64 (got %d)", rope_dims);
+  *bytes = swa_ws(Tq, kv_len, Hq, d, rope_dims).total;
+  return HS2_OK;
+}
+
+hs2_status hs2_swa_attn_prefill(const void* Q, const void* K, const void* V, int64_t q_start, int64_t Tq,
+                                int64_t kv_len, int Hq, int d, int window, int rope_dims, float rope_base,
+                                float softmax_scale, void* O, void* workspace, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(Q && K && V && O, HS2_ERR_INVALID_ARG, "null tensor pointer");
+  HS2_CHECK(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O), HS2_ERR_INVALID_ARG,
+            "tensor pointers must be 16-byte aligned");
+  HS2_CHECK(Tq >= 1 && kv_len >= 1 && q_start >= 0 && q_start + Tq <= kv_len, HS2_ERR_INVALID_ARG,
+            "bad sizes (need q_start + Tq <= kv_len)");
+  HS2_CHECK(Tq * Hq < (1ll << 31) && kv_len < (1ll << 31), HS2_ERR_UNSUPPORTED, "sizes beyond int32 tiles");
+  HS2_CHECK(window >= 1, HS2_ERR_INVALID_ARG, "window must be >= 1");
+  HS2_CHECK(std::isfinite(rope_base) && rope_base > 1.f, HS2_ERR_INVALID_ARG, "rope_base must be > 1");
+  HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  size_t need = 0;
+  hs2_status s = hs2_swa_attn_prefill_workspace(Tq, kv_len, Hq, d, rope_dims, &need);
+  if (s != HS2_OK) return s;
+  HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) && ws_bytes >= need,
+            HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
+  DevCtx ctx;
+  if ((s = device_ctx(&ctx, nullptr)) != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? swa_attn<256>(Q, K, V, q_start, Tq, kv_len, Hq, window, rope_dims, rope_base, softmax_scale, O,
+                                  workspace, st, ctx)
+                  : swa_attn<128>(Q, K, V, q_start, Tq, kv_len, Hq, window, rope_dims, rope_base, softmax_scale, O,
+                                  workspace, st, ctx);
 }
 
 hs2_status hs2_device_status(void* stream) {
