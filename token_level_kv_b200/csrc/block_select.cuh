@@ -16,7 +16,8 @@
 // as the token-level path.  The scores of a row are summed per block in a
 // fixed order (each of G = min(B, 32) lanes adds B/G scores, then a shuffle
 // tree), so a block score carries at most B/G - 1 + log2(G) roundings; the
-// block scores (at most 16384 per row) stay in shared memory, where an exact
+// block scores (at most 16384 per row; shared memory is sized to the call's
+// longest row) stay in shared memory, where an exact
 // 4-pass radix select over their fp32 bit patterns (scores are >= 0, so the
 // patterns order like the values) finds the k-th largest; two block-wide
 // scans then mark the ties taken and place each chosen block's positions.
@@ -27,7 +28,8 @@ namespace hs2 {
 
 constexpr int BS_THREADS = 256;
 constexpr int BS_MAX_BLOCKS = 16384;
-constexpr size_t BS_SMEM = (size_t)BS_MAX_BLOCKS * 4 + 256 * 4;
+// shared memory for rows of at most nb_max blocks: the block scores, then 256 bins
+__host__ __device__ constexpr size_t bs_smem(int nb_max) { return ((size_t)nb_max + 256) * 4; }
 
 struct BlockSelParams {
   const float* sigma;    // row r at sigma + r * ld, candidates [0, n_r)
@@ -37,6 +39,7 @@ struct BlockSelParams {
   int window;
   int block;             // B: a power of two in [16, 256]
   int topk_blocks;       // k
+  int nb_max;            // the most blocks any row has (sizes shared memory)
   int32_t* idx;          // [rows, window + k * B]
 };
 
@@ -67,7 +70,7 @@ __global__ void __launch_bounds__(BS_THREADS)
 block_select_kernel(BlockSelParams p, DevCtx ctx) {
   extern __shared__ __align__(16) uint8_t smem_bs[];
   uint32_t* bsc = reinterpret_cast<uint32_t*>(smem_bs);               // block scores (fp32 patterns)
-  uint32_t* hist = bsc + BS_MAX_BLOCKS;                               // 256 bins
+  uint32_t* hist = bsc + p.nb_max;                                    // 256 bins
   __shared__ uint32_t scratch[BS_THREADS / 32];
   __shared__ uint32_t pick[2];                                         // chosen bin, count above it
 
@@ -91,25 +94,33 @@ block_select_kernel(BlockSelParams p, DevCtx ctx) {
   const int per_lane = B / G;
   const int bpw = 32 / G;                                              // blocks per warp step
   const int sub = lane / G, gl = lane % G;
-  for (int c0 = warp * bpw; c0 < nb; c0 += (BS_THREADS / 32) * bpw) {
-    const int c = c0 + sub;
-    float acc = 0.f;
-    if (c < nb) {
+  // four block steps of a warp at a time, their loads issued together
+  constexpr int U = 4;
+  bool bad = false;
+  for (int c0 = warp * bpw; c0 < nb; c0 += (BS_THREADS / 32) * bpw * U) {
+    float acc[U];
+#pragma unroll
+    for (int s = 0; s < U; ++s) {
+      const int c = c0 + s * (BS_THREADS / 32) * bpw + sub;
+      acc[s] = 0.f;
       for (int i = 0; i < per_lane; ++i) {
         const int64_t j = (int64_t)c * B + (int64_t)i * G + gl;
-        if (j < n) {
+        if (c < nb && j < n) {
           uint32_t u = __float_as_uint(src[j]);
-          if (u > 0x7f800000u) {                                       // NaN or negative: not a probability sum
-            report(ctx, ST_DEVICE_CHECK);
-            u = 0u;
-          }
-          acc += __uint_as_float(u);
+          bad |= u > 0x7f800000u;                                      // NaN or negative: not a probability sum
+          acc[s] += __uint_as_float(u > 0x7f800000u ? 0u : u);
         }
       }
     }
-    for (int o = G / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (gl == 0 && c < nb) bsc[c] = __float_as_uint(acc);
+#pragma unroll
+    for (int s = 0; s < U; ++s) {
+      const int c = c0 + s * (BS_THREADS / 32) * bpw + sub;
+      float a = acc[s];
+      for (int o = G / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (gl == 0 && c < nb) bsc[c] = __float_as_uint(a);
+    }
   }
+  if (bad) report(ctx, ST_DEVICE_CHECK);
   __syncthreads();
 
   // ---- the k-th largest pattern T and how many blocks equal to T are taken
@@ -161,32 +172,39 @@ block_select_kernel(BlockSelParams p, DevCtx ctx) {
   }
 
   // ---- mark (ties taken in block order) and place: thread t owns blocks
-  // [t*per, (t+1)*per)
-  const int per = (nb + BS_THREADS - 1) / BS_THREADS;
+  // [t*per, (t+1)*per), per odd so a warp's 32 lanes hit 32 banks
+  const int per = ((nb + BS_THREADS - 1) / BS_THREADS) | 1;
   const int c0 = threadIdx.x * per, c1 = min(nb, c0 + per);
   uint32_t n_eq = 0;
   for (int c = c0; c < c1; ++c) n_eq += bsc[c] == T ? 1u : 0u;
   uint32_t tot;
   uint32_t eq_before = bs_excl_scan(n_eq, scratch, tot);
-  uint32_t n_pos = 0;
+  // the chosen blocks, in block order, into sel[]: every chosen block but a
+  // partial last one holds B positions, and a partial block is the last
+  // block of the row, so chosen block r starts at slot r * B
+  uint32_t n_take = 0;
   for (int c = c0; c < c1; ++c) {
     const uint32_t u = bsc[c];
     bool take = u > T;
     if (u == T) take = eq_before++ < need_eq;
-    if (take) n_pos += (uint32_t)min((int64_t)B, n - (int64_t)c * B);
+    n_take += take ? 1u : 0u;
     bsc[c] = take ? 1u : 0u;                                          // own blocks only: no race
   }
-  uint32_t at = bs_excl_scan(n_pos, scratch, tot);
-  for (int c = c0; c < c1; ++c) {
-    if (!bsc[c]) continue;
-    const int64_t j1 = min(n, (int64_t)(c + 1) * B);
-    for (int64_t j = (int64_t)c * B; j < j1; ++j) {
-      if (at < (uint32_t)(k * B)) out[W + at] = (int32_t)j;
-      ++at;
-    }
+  uint32_t n_sel;
+  uint32_t rank = bs_excl_scan(n_take, scratch, n_sel);
+  uint32_t* sel = hist;                                               // the bins are free again
+  for (int c = c0; c < c1; ++c)
+    if (bsc[c] && rank < (uint32_t)k) sel[rank++] = (uint32_t)c;
+  __syncthreads();
+  // one warp per chosen block: its positions, lanes on consecutive slots
+  const uint32_t n_blk = min(n_sel, (uint32_t)k);
+  for (uint32_t r = warp; r < n_blk; r += BS_THREADS / 32) {
+    const int64_t j0 = (int64_t)sel[r] * B;
+    const int len = (int)min((int64_t)B, n - j0);
+    for (int i = lane; i < B; i += 32) out[W + (int64_t)r * B + i] = i < len ? (int32_t)(j0 + i) : -1;
   }
-  for (uint32_t i = tot + threadIdx.x; i < (uint32_t)(k * B); i += BS_THREADS) out[W + i] = -1;
-  if (threadIdx.x == 0 && tot > (uint32_t)(k * B)) report(ctx, ST_DEVICE_CHECK);
+  for (int i = n_blk * B + threadIdx.x; i < k * B; i += BS_THREADS) out[W + i] = -1;
+  if (threadIdx.x == 0 && n_sel > (uint32_t)k) report(ctx, ST_DEVICE_CHECK);
 }
 
 }  // namespace hs2
