@@ -309,25 +309,54 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
 
 // Merge split partials of one (item, head) per CTA, one output dim per
 // thread: m = max m_s, l = sum l_s 2^(m_s-m), O = sum O_s 2^(m_s-m) / l.
-// Also stores (m, l) per head (log2 units) for the selection pass.
+// Also stores (m, l) per head (log2 units) for the selection pass.  The
+// split factors are computed once, cooperatively, into shared memory, so the
+// O loop's loads are independent of one another (a full-attention pass over
+// 2^20 keys has 512 splits per sequence).
+constexpr int kCombineMaxSplits = 1024;
 template <int D>
 __global__ void __launch_bounds__(D)
 attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, float* ml) {
   const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
-  const float* base = part + (int64_t)item * splits * (32 + 16 * D);
+  const int lane = c & 31, warp = c >> 5;
+  constexpr int PS = 32 + 16 * D;                   // floats per partial
+  __shared__ float fac[kCombineMaxSplits];
+  __shared__ float red[D / 32];
+  const float* base = part + (int64_t)item * splits * PS;
   float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, base[s * (32 + 16 * D) + h]);
-  float Ls = 0.f, acc = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float* ps = base + s * (32 + 16 * D);
-      const float ms = ps[h];
-      if (ms == -INFINITY) continue;
-      const float f = fast_exp2(ms - M);
-      Ls += ps[16 + h] * f;
-      acc += ps[32 + h * D + c] * f;
-    }
+  for (int s = c; s < splits; s += D) M = fmaxf(M, base[(int64_t)s * PS + h]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  float ls = 0.f;
+  for (int s = c; s < splits; s += D) {
+    const float ms = base[(int64_t)s * PS + h];
+    const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
+    fac[s] = f;
+    ls += base[(int64_t)s * PS + 16 + h] * f;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane == 0) red[warp] = ls;
+  __syncthreads();
+  float Ls = 0.f;
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) Ls += red[w];
+  const float* col = base + 32 + h * D + c;
+  float acc0 = 0.f, acc1 = 0.f;
+  int s = 0;
+#pragma unroll 4
+  for (; s + 1 < splits; s += 2) {
+    acc0 += col[(int64_t)s * PS] * fac[s];
+    acc1 += col[(int64_t)(s + 1) * PS] * fac[s + 1];
+  }
+  if (s < splits) acc0 += col[(int64_t)s * PS] * fac[s];
+  const float acc = acc0 + acc1;
   if (c == 0 && ml != nullptr) {
     ml[((int64_t)item * H + h) * 2] = M;
     ml[((int64_t)item * H + h) * 2 + 1] = Ls;

@@ -281,6 +281,7 @@ int sparse_decode_splits(int batch, int n_idx, int num_sms) {
 template <int D>
 hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
                           cudaStream_t st) {
+  if (splits > kCombineMaxSplits) return fail(HS2_ERR_UNSUPPORTED, "%d split partials (at most %d)", splits, kCombineMaxSplits);
   prof_begin(st);
   attn16_combine_kernel<D><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml);
   return after_launch("attn16_combine_kernel", st);
