@@ -182,19 +182,24 @@ select_sigma_kernel(const __grid_constant__ CUtensorMap tmQ256, const __grid_con
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, ctx))) break;
       tc_fence_after();
       const int64_t key = (int64_t)j * 128 + kl;
-#pragma unroll 1
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        float v[32];
+      // four chunks of 16 columns; chunk c+1's TMEM load is in flight while
+      // chunk c is computed (tcgen05.wait::ld waits for all of this thread's
+      // loads, so the next one is issued right after the wait)
+      const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+      float va[16], vb[16];
+      tmem_ld16(lane_base + buf * 256 + part * 64, va);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) tmem_ld16(lane_base + buf * 256 + part * 64 + c0 + c * 16, v + c * 16);
+      for (int ch = 0; ch < 4; ++ch) {
+        float* v = (ch & 1) ? vb : va;
+        float* nxt = (ch & 1) ? va : vb;
         tmem_wait_ld();
-        // column part*64 + c0 + i  <->  (query (part*64 + c0 + i) / H, head i % H);
+        if (ch < 3) tmem_ld16(lane_base + buf * 256 + part * 64 + (ch + 1) * 16, nxt);
+        // column part*64 + 16*ch + i  <->  (query (part*64 + 16*ch + i) / H, head i % H);
         // heads in pairs: one packed FMA for the two exponents' arguments and
         // one for the two terms of the sum (two interleaved partial sums)
-        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
-        for (int qi = 0; qi < 32 / H; ++qi) {
-          const int col = part * 64 + c0 + qi * H;
+        for (int qi = 0; qi < 16 / H; ++qi) {
+          const int col = part * 64 + ch * 16 + qi * H;
           const int64_t tq = g0 + col / H;
           const int64_t pq = p.q_start + tq;
           uint64_t acc2 = 0ull;
