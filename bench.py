@@ -379,6 +379,8 @@ def run_ours(args, rank, world, dist):
     sel_ms = sum(kern.get(n, {"avg_ms": 0.0})["avg_ms"] for n in ("fa_fwd_kernel", "select_sigma_kernel",
                                                                   "topk_select_kernel"))
     sel_ach = full_fl / (sel_ms * 1e-3) / 1e12 if sel_ms > 0 else None
+    # ---------------- the same call with block-level selection (64-token blocks, 16 of them)
+    blocks = bench_select_blocks(hs2, case, ws, flush, stream, full_fl, peaks) if not args.no_blocks else None
     stages = {n: {"avg_ms": v["avg_ms"], "launches": v["launches"], "share": v["total_ms"] / sum(
         x["total_ms"] for x in kern.values())} for n, v in kern.items()}
 
@@ -395,6 +397,7 @@ def run_ours(args, rank, world, dist):
                         "algorithmic_flops": full_fl, "executed_extra_flops_sigma_pass": sigma_fl,
                         "unit": "TFLOP/s", "peak": peaks["bf16_tflops"]},
         "stages": stages,
+        "select_blocks": blocks,
         "gpu_launches": launches,
         "wall_s_timed_region": t_wall,
     }
@@ -467,6 +470,7 @@ def run_ours(args, rank, world, dist):
         out["prefill_256k"] = bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args)
         torch.cuda.empty_cache()
     out["prefill_1k"] = bench_tiny(hs2, dev, stream, flush, args)
+    out["swa_32k"] = bench_swa(hs2, case, flush, stream, peaks)
     out["select_call_frac"] = {"prefill_32k": out["select_call"]["frac"],
                                "prefill_256k_chunked": out.get("prefill_256k", {}).get("select_call_frac"),
                                "peak": f"{peak_src} bf16_tflops", "target": 0.60}
@@ -558,6 +562,32 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
     }
 
 
+def bench_select_blocks(hs2, case, ws, flush, stream, full_fl, peaks, block=64, topk_blocks=16):
+    """The full-attention layer with block-level selection on the same inputs:
+    aligned 64-token blocks scored by their summed selection scores, the top
+    16 taken (the pages' token-vs-block ablation at the same 1024 budget)."""
+    T, H, d = case.Q.shape
+    W = WORKLOAD["window"]
+    O = torch.empty(T, H, d, dtype=torch.bfloat16, device=case.Q.device)
+    idx = torch.empty(T, W + block * topk_blocks, dtype=torch.int32, device=case.Q.device)
+
+    def call():
+        hs2.hs2_full_attn_select_blocks(case.Q, case.K, case.V, O, idx, ws, window=W, block=block,
+                                        topk_blocks=topk_blocks)
+
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    hs2.hs2_profile_enable(True)
+    t = timed_steps(call, 3, flush, stream)
+    prof = per_kernel(hs2.hs2_profile_collect())
+    hs2.hs2_profile_enable(False)
+    ms = statistics.median(t)
+    return {"workload": f"as the step's full layer, block-level selection: {topk_blocks} blocks of {block} tokens",
+            "ms": ms, "frac": full_fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "kernels": {k: v["avg_ms"] for k, v in prof.items()}}
+
+
 def bench_bridge(hs2, dev, stream, flush, peaks, peak_src):
     """KV Bridging of 4 x 2^20 hidden rows into 2 layers' FP8 caches; returns
     the result and the caches (the bridged decode step reads them)."""
@@ -602,7 +632,8 @@ def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged
     import synth
     caches, hid_new, weights = bridged
     c = synth.CONFIGS[5]
-    B, N, H, d, W, k, ns = c["B"], c["N"], c["H"], c["d"], c["window"], c["topk"], c["n_sparse"]
+    B, H, d, W, k, ns = c["B"], c["H"], c["d"], c["window"], c["topk"], c["n_sparse"]
+    N = BRIDGE["R"] // B                          # tokens per sequence of the bridged caches
     qs = synth.bridged_decode_queries(B, H, d, len(caches), ns, seed=0, device=dev)
     O = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
     Os = torch.empty_like(O)
@@ -693,6 +724,31 @@ def bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args):
     return res
 
 
+def bench_swa(hs2, case, flush, stream, peaks, window=128):
+    """A self-decoder sliding-window layer at the prefill head shape (the
+    step's Q, K, V; window 128, 64-dim partial RoPE)."""
+    T, H, d = case.Q.shape
+    O = torch.empty_like(case.Q)
+    ws = hs2.workspace(hs2.hs2_swa_attn_prefill_workspace(T, T, H, d), case.Q.device)
+
+    def call():
+        hs2.hs2_swa_attn_prefill(case.Q, case.K, case.V, O, ws, window=window)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    hs2.hs2_profile_enable(True)
+    t = timed_steps(call, 5, flush, stream)
+    prof = per_kernel(hs2.hs2_profile_collect())
+    hs2.hs2_profile_enable(False)
+    ms = statistics.median(t)
+    pairs = sum(min(p + 1, window) for p in range(T))
+    fl = 4.0 * d * H * pairs
+    return {"workload": f"sliding-window attention T={T} H={H} d={d}, window {window}, 64-dim partial RoPE",
+            "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_flops": fl,
+            "kernels": {k: v["avg_ms"] for k, v in prof.items()}}
+
+
 def bench_tiny(hs2, dev, stream, flush, args):
     """The tiny single-sequence case (T = 1024, 8 heads, d = 128, window 128 +
     top-256, 1 sparse layer): launch-bound, reported only."""
@@ -734,6 +790,9 @@ def main():
     ap.add_argument("--no-bridge", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the 256k chunked prefill")
+    ap.add_argument("--no-blocks", action="store_true", help="skip the block-level selection call")
+    ap.add_argument("--bridge-rows", type=int, default=None,
+                    help="override the bridged workload's rows, 4 sequences of rows/4 tokens (small profiling cases)")
     ap.add_argument("--long-T", type=int, default=None, help="override the chunked prefill length (small profiling cases)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=48)
@@ -747,6 +806,8 @@ def main():
         DECODE["N"] = args.decode_N
     if args.decode_B:
         DECODE["B"] = args.decode_B
+    if args.bridge_rows:
+        BRIDGE["R"] = args.bridge_rows
     if args.T:
         WORKLOAD["T"] = args.T
         WORKLOAD["n_needles"] = min(WORKLOAD["n_needles"], max(0, args.T // 512))

@@ -274,6 +274,104 @@ HS2_API hs2_status hs2_swa_attn_prefill_workspace(int64_t Tq, int64_t kv_len, in
                                                   int rope_dims, size_t* bytes);
 
 /*
+ * Decode with each sequence's context split over R shards (one per GPU), for
+ * the 1M-token regime with few sequences (agihunt.info summary, KV cache
+ * table at 1M tokens; the selection and reuse are those of
+ * hs2_full_attn_select and hs2_sparse_attn_decode).  Shard q holds the
+ * positions [offset_q, offset_q + shard_len_q) of every sequence, offsets
+ * ascending with q and the shards tiling [0, kv_len).  One decode step of a
+ * full-attention layer and its sparse layers, on every shard:
+ *   1. hs2_decode_shard_attn: full attention over the shard -> (m, l) and an
+ *      unnormalised O; the shard's logits stay in the workspace.
+ *   2. exchange: all-gather the R (m, l) blocks -> ml_all [R][2][batch, Hq].
+ *   3. hs2_partial_merge: global (M, L) per head -> ml_global [batch, Hq, 2],
+ *      this shard's O rescaled to M.
+ *   4. exchange: sum-all-reduce O32 over the shards.
+ *   5. hs2_partial_finalize: O = O32 / L (bf16), the full-attention output.
+ *   6. hs2_decode_shard_candidates: selection scores of the shard's
+ *      candidates under the global (M, L), the shard's top-k as a list.
+ *   7. exchange: all-gather the lists -> cand_all [R][...].
+ *   8. hs2_decode_merge_candidates: the index row [batch, window + topk],
+ *      identical to hs2_full_attn_select's on the whole cache.
+ *   9. per sparse layer: hs2_sparse_decode_shard (the index entries that fall
+ *      in the shard), then steps 2-5 again for that layer's output.
+ * The exchanges are the caller's (e.g. NCCL through torch.distributed).
+ * Results equal the single-GPU calls' up to the order of fp32 additions.
+ *
+ * hs2_decode_shard_attn:
+ *   Q bf16 [batch, Hq, d]; Kc, Vc uint8 [batch, kv_stride_tokens, d] and
+ *   k_scale, v_scale fp32 [batch, kv_stride_tokens]: the shard's part of the
+ *   FP8 cache, local position i = global position offset + i, i < shard_len.
+ *   ml_out fp32 [2][batch, Hq]: m (the max of the scaled logits, log2 units)
+ *   then l (the sum of 2^(logit - m)); -inf and 0 for no key.
+ *   O_out fp32 [batch, Hq, d]: sum_j 2^(logit_j - m) v_j, not normalised.
+ *   workspace: hs2_decode_shard_workspace() bytes, 256-byte aligned; it must
+ *   be kept, unchanged, for hs2_decode_shard_candidates of the same step.
+ *   topk only sizes the workspace; pass the step's topk.
+ */
+HS2_API hs2_status hs2_decode_shard_workspace(int batch, int64_t shard_len, int n_idx, int Hq, int d,
+                                              int topk, size_t* bytes);
+
+HS2_API hs2_status hs2_decode_shard_attn(const void* Q, const void* Kc, const void* Vc,
+                                         const float* k_scale, const float* v_scale, int batch,
+                                         int64_t shard_len, int64_t kv_stride_tokens, int Hq, int d,
+                                         int topk, float softmax_scale, float* ml_out, float* O_out,
+                                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * ml_all fp32 [n_shards][2][batch, Hq] (every shard's ml_out, shard order);
+ * O32 fp32 [batch, Hq, d]: shard `shard`'s O, rescaled in place by
+ * 2^(m_shard - M); ml_out fp32 [batch, Hq, 2]: (M, L) with M = max m and
+ * L = sum_q l_q 2^(m_q - M), the same on every shard.
+ */
+HS2_API hs2_status hs2_partial_merge(const float* ml_all, int n_shards, int shard, float* O32,
+                                     float* ml_out, int batch, int Hq, int d, void* stream);
+
+/* O bf16 [batch, Hq, d] = O32 / L, with ml = (M, L) [batch, Hq, 2]; 0 where L = 0. */
+HS2_API hs2_status hs2_partial_finalize(const float* ml, const float* O32, void* O, int batch, int Hq,
+                                        int d, void* stream);
+
+/*
+ * The shard's candidates are the global positions offset .. kv_len-1-window
+ * that it holds; their selection scores sigma_j = sum_h 2^(logit_hj - M_h)/L_h
+ * use the logits hs2_decode_shard_attn left in `workspace` and
+ * ml_global = (M, L) from hs2_partial_merge.  cand (4-byte elements):
+ * scores fp32 [batch, topk], then global positions int32 [batch, topk], then
+ * list lengths int32 [batch]; a row's list is its top min(topk, n) candidates
+ * in ascending position (the order of hs2_full_attn_select: score
+ * descending, ties to the smaller position).
+ */
+HS2_API hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int batch,
+                                               int64_t shard_len, int64_t shard_offset, int64_t kv_len,
+                                               int Hq, int d, int window, int topk,
+                                               const float* ml_global, void* cand, void* stream);
+
+/*
+ * cand_all: n_shards (<= 64) blocks of hs2_decode_shard_candidates' cand,
+ * shard order.  idx int32 [batch, window + topk]: the window positions
+ * kv_len-window .. kv_len-1 (-1 below 0), then the top-k of all lists in
+ * ascending position, -1 padded.
+ */
+HS2_API hs2_status hs2_decode_merge_candidates(const void* cand_all, int n_shards, int batch,
+                                               int64_t kv_len, int window, int topk, int32_t* idx,
+                                               void* stream);
+
+/*
+ * A sparse layer's decode over one shard: hs2_sparse_attn_decode restricted
+ * to the entries of idx (global positions) in [shard_offset,
+ * shard_offset + shard_len), with the partial outputs of
+ * hs2_decode_shard_attn (ml_out [2][batch, Hq], O_out fp32 [batch, Hq, d]).
+ * The cache arguments are the shard's, as in hs2_decode_shard_attn.
+ * workspace: hs2_decode_shard_workspace() bytes with this n_idx.
+ */
+HS2_API hs2_status hs2_sparse_decode_shard(const void* Q, const void* Kc, const void* Vc,
+                                           const float* k_scale, const float* v_scale, int batch,
+                                           int64_t shard_len, int64_t kv_stride_tokens,
+                                           int64_t shard_offset, const int32_t* idx, int n_idx, int Hq,
+                                           int d, float softmax_scale, float* ml_out, float* O_out,
+                                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the status word of the current
  * device: HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA if
  * the synchronisation itself failed).

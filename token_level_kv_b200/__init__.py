@@ -52,6 +52,13 @@ def _load() -> ctypes.CDLL:
         "hs2_sparse_attn_decode_static": ([P, P, P, P, P, I, I, L, L, P, I, I, I, F, P, P], I),
         "hs2_swa_attn_prefill": ([P, P, P, L, L, L, I, I, I, I, F, F, P, P, Z, P], I),
         "hs2_swa_attn_prefill_workspace": ([L, L, I, I, I, ctypes.POINTER(Z)], I),
+        "hs2_decode_shard_workspace": ([I, L, I, I, I, I, ctypes.POINTER(Z)], I),
+        "hs2_decode_shard_attn": ([P, P, P, P, P, I, L, L, I, I, I, F, P, P, P, Z, P], I),
+        "hs2_partial_merge": ([P, I, I, P, P, I, I, I, P], I),
+        "hs2_partial_finalize": ([P, P, P, I, I, I, P], I),
+        "hs2_decode_shard_candidates": ([P, Z, I, L, L, L, I, I, I, I, P, P, P], I),
+        "hs2_decode_merge_candidates": ([P, I, I, L, I, I, P, P], I),
+        "hs2_sparse_decode_shard": ([P, P, P, P, P, I, L, L, L, P, I, I, I, F, P, P, P, Z, P], I),
         "hs2_device_status": ([P], I),
         "hs2_set_spin_limit": ([L], I),
         "hs2_profile_enable": ([I], I),
@@ -69,7 +76,9 @@ EXPORTS = ("hs2_status_string", "hs2_last_error", "hs2_version", "hs2_bridge_kv"
            "hs2_full_attn_select_workspace", "hs2_sparse_attn_prefill", "hs2_sparse_attn_decode",
            "hs2_sparse_attn_decode_workspace", "hs2_device_status", "hs2_set_spin_limit",
            "hs2_profile_enable", "hs2_profile_collect", "hs2_sparse_attn_decode_static", "hs2_bridge_append",
-           "hs2_full_attn_select_blocks", "hs2_swa_attn_prefill", "hs2_swa_attn_prefill_workspace")
+           "hs2_full_attn_select_blocks", "hs2_swa_attn_prefill", "hs2_swa_attn_prefill_workspace",
+           "hs2_decode_shard_workspace", "hs2_decode_shard_attn", "hs2_partial_merge", "hs2_partial_finalize",
+           "hs2_decode_shard_candidates", "hs2_decode_merge_candidates", "hs2_sparse_decode_shard")
 
 
 def _check(status: int) -> None:
@@ -241,6 +250,78 @@ def hs2_sparse_attn_decode_static(Q, Kc, Vc, k_scale, v_scale, idx, O, *, kv_len
     _check(lib.hs2_sparse_attn_decode_static(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale),
                                              KV_FP8_E4M3, B, kv_len, stride, _ptr(idx), idx.shape[-1], H, d,
                                              scale, _ptr(O), _stream(stream)))
+
+
+# ---- decode with the context split over shards (one per GPU); the exchanges
+# between the calls are the caller's (token_level_kv_b200.sharded runs them
+# over torch.distributed)
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def hs2_decode_shard_workspace(batch: int, shard_len: int, n_idx: int, Hq: int, d: int, topk: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hs2_decode_shard_workspace(batch, shard_len, n_idx, Hq, d, topk, ctypes.byref(n)))
+    return n.value
+
+
+def candidates_numel(batch: int, topk: int) -> int:
+    """4-byte elements of one shard's candidate block: scores, positions, lengths."""
+    return 2 * batch * topk + batch
+
+
+def hs2_decode_shard_attn(Q, Kc, Vc, k_scale, v_scale, ml_out, O_out, workspace, *, topk: int,
+                          shard_len: int | None = None, softmax_scale: float | None = None, stream=None) -> None:
+    """Full attention over one shard: ml_out fp32 [2, B, H] (m, l), O_out fp32 [B, H, d] unnormalised."""
+    B, H, d = Q.shape
+    stride = Kc.shape[1]
+    n = stride if shard_len is None else shard_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    _check(lib.hs2_decode_shard_attn(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale), B, n, stride, H,
+                                     d, topk, scale, _ptr(ml_out), _ptr(O_out), _ptr(workspace),
+                                     _nbytes(workspace), _stream(stream)))
+
+
+def hs2_partial_merge(ml_all, shard: int, O32, ml_out, stream=None) -> None:
+    """ml_all fp32 [R, 2, B, H]; rescales O32 [B, H, d] in place; ml_out fp32 [B, H, 2] = (M, L)."""
+    R, _, B, H = ml_all.shape
+    _check(lib.hs2_partial_merge(_ptr(ml_all), R, shard, _ptr(O32), _ptr(ml_out), B, H, O32.shape[-1],
+                                 _stream(stream)))
+
+
+def hs2_partial_finalize(ml, O32, O, stream=None) -> None:
+    """O bf16 [B, H, d] = O32 / L."""
+    B, H, d = O32.shape
+    _check(lib.hs2_partial_finalize(_ptr(ml), _ptr(O32), _ptr(O), B, H, d, _stream(stream)))
+
+
+def hs2_decode_shard_candidates(workspace, ml_global, cand, *, batch: int, shard_len: int, shard_offset: int,
+                                kv_len: int, Hq: int, d: int, window: int, topk: int, stream=None) -> None:
+    """The shard's top-k candidates under the global (M, L) into cand (candidates_numel 4-byte elements)."""
+    _check(lib.hs2_decode_shard_candidates(_ptr(workspace), _nbytes(workspace), batch, shard_len, shard_offset,
+                                           kv_len, Hq, d, window, topk, _ptr(ml_global), _ptr(cand),
+                                           _stream(stream)))
+
+
+def hs2_decode_merge_candidates(cand_all, idx, *, kv_len: int, window: int, topk: int, stream=None) -> None:
+    """cand_all [R, candidates_numel]; idx int32 [B, window + topk]."""
+    R = cand_all.shape[0]
+    B = idx.shape[0]
+    _check(lib.hs2_decode_merge_candidates(_ptr(cand_all), R, B, kv_len, window, topk, _ptr(idx), _stream(stream)))
+
+
+def hs2_sparse_decode_shard(Q, Kc, Vc, k_scale, v_scale, idx, ml_out, O_out, workspace, *, shard_offset: int,
+                            shard_len: int | None = None, softmax_scale: float | None = None,
+                            stream=None) -> None:
+    """A sparse layer over one shard: the entries of idx (global positions) the shard holds."""
+    B, H, d = Q.shape
+    stride = Kc.shape[1]
+    n = stride if shard_len is None else shard_len
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    _check(lib.hs2_sparse_decode_shard(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(k_scale), _ptr(v_scale), B, n, stride,
+                                       shard_offset, _ptr(idx), idx.shape[-1], H, d, scale, _ptr(ml_out),
+                                       _ptr(O_out), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def hs2_device_status(stream=None) -> int:

@@ -314,9 +314,11 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
 // O loop's loads are independent of one another (a full-attention pass over
 // 2^20 keys has 512 splits per sequence).
 constexpr int kCombineMaxSplits = 1024;
+// With O32 set, the merged O is written unnormalised (fp32, relative to m) for
+// a later merge across shards of the context, and O is not written.
 template <int D>
 __global__ void __launch_bounds__(D)
-attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, float* ml) {
+attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, float* O32) {
   const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
   const int lane = c & 31, warp = c >> 5;
   constexpr int PS = 32 + 16 * D;                   // floats per partial
@@ -358,10 +360,56 @@ attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, fl
   if (s < splits) acc0 += col[(int64_t)s * PS] * fac[s];
   const float acc = acc0 + acc1;
   if (c == 0 && ml != nullptr) {
-    ml[((int64_t)item * H + h) * 2] = M;
-    ml[((int64_t)item * H + h) * 2 + 1] = Ls;
+    const int64_t r = (int64_t)item * H + h;
+    if (O32 != nullptr) {                           // a shard's partial: m, then l, each [items, H]
+      ml[r] = M;
+      ml[(int64_t)gridDim.x * H + r] = Ls;
+    } else {
+      ml[r * 2] = M;
+      ml[r * 2 + 1] = Ls;
+    }
   }
-  O[((int64_t)item * H + h) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
+  if (O32 != nullptr) O32[((int64_t)item * H + h) * D + c] = acc;
+  else O[((int64_t)item * H + h) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
+}
+
+// Merge of partials across the R shards of a context.  ml_all holds every
+// shard's (m, l) as [R][2][items * H] (m in log2 units; an all-gather of
+// each shard's planar (m, l) gives it); for each (item, head) the kernel takes
+// M = max_q m_q and L = sum_q l_q 2^(m_q - M), rescales this shard's
+// unnormalised O by 2^(m_shard - M) (0 for a shard that saw no key), so that
+// the shards' O then add up, and writes (M, L) interleaved to ml_out.  Every
+// shard computes the same M and L in the same order.
+template <int D>
+__global__ void __launch_bounds__(D)
+partial_merge_kernel(const float* ml_all, int R, int shard, float* O32, float* ml_out, int H) {
+  const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  const int64_t n = (int64_t)gridDim.x * H;
+  const int64_t r = (int64_t)item * H + h;
+  float M = -INFINITY;
+  for (int q = 0; q < R; ++q) M = fmaxf(M, ml_all[q * 2 * n + r]);
+  float L = 0.f;
+  for (int q = 0; q < R; ++q) {
+    const float m = ml_all[q * 2 * n + r];
+    L += (m == -INFINITY) ? 0.f : ml_all[q * 2 * n + n + r] * fast_exp2(m - M);
+  }
+  const float m = ml_all[shard * 2 * n + r];
+  const float f = m == -INFINITY ? 0.f : fast_exp2(m - M);
+  O32[r * D + c] *= f;
+  if (c == 0) {
+    ml_out[r * 2] = M;
+    ml_out[r * 2 + 1] = L;
+  }
+}
+
+// The merged output: O = (sum of the shards' rescaled O) / (sum of their l).
+template <int D>
+__global__ void __launch_bounds__(D)
+partial_finalize_kernel(const float* ml, const float* O32, __nv_bfloat16* O, int H) {
+  const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  const int64_t r = (int64_t)item * H + h;
+  const float l = ml[r * 2 + 1];
+  O[r * D + c] = __float2bfloat16_rn(l > 0.f ? O32[r * D + c] / l : 0.f);
 }
 
 // Decode selection score: sigma[b, j] = sum_h 2^(x_hj - m_h) / l_h for the

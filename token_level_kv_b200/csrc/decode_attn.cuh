@@ -129,6 +129,8 @@ struct DecParams {
   int splits;               // CTAs per sequence
   int per_split;            // keys (range) or idx slots (gather) per CTA
   __nv_bfloat16* O;         // [B, H, D] (gather)
+  int64_t idx_offset;       // gather over one shard of the context: idx entries are global positions and
+                            // only [idx_offset, idx_offset + kv_len) are this shard's (rebased); -1: no shard
   float* part;              // [B, splits, 32 + 16*D] (range)
   float* logits;            // [B, H, logit_ld] (range)
   int64_t logit_ld;
@@ -200,7 +202,10 @@ decode_attn_kernel(DecParams p, DevCtx ctx, const __grid_constant__ CUtensorMap 
   if (!RANGE) {
     for (int64_t i = threadIdx.x; i < s_end - s_begin; i += blockDim.x) {
       const int32_t v = sidx[i];
-      if (v < -1 || v >= p.kv_len) {
+      if (p.idx_offset >= 0) {                       // a shard: other shards' keys are not errors
+        sidx[i] = (v >= p.idx_offset && v < p.idx_offset + p.kv_len) ? (int32_t)(v - p.idx_offset) : -1;
+        if (v < -1) report(ctx, ST_DEVICE_CHECK);
+      } else if (v < -1 || v >= p.kv_len) {
         report(ctx, ST_DEVICE_CHECK);
         sidx[i] = -1;
       }

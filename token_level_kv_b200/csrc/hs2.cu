@@ -280,10 +280,10 @@ int sparse_decode_splits(int batch, int n_idx, int num_sms) {
 // ------------------------------------------------------------------ launches
 template <int D>
 hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, int items,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* O32 = nullptr) {
   if (splits > kCombineMaxSplits) return fail(HS2_ERR_UNSUPPORTED, "%d split partials (at most %d)", splits, kCombineMaxSplits);
   prof_begin(st);
-  attn16_combine_kernel<D><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml);
+  attn16_combine_kernel<D><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml, O32);
   return after_launch("attn16_combine_kernel", st);
 }
 
@@ -460,6 +460,7 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   p.part = part;
   p.logits = logits;
   p.logit_ld = w.ld;
+  p.idx_offset = -1;
   using L = DecLayout<D, true>;
   auto k = decode_attn_kernel<D, true, true>;
   hs2_status s = set_smem(k, L::SMEM);
@@ -484,7 +485,7 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   }
   if (block == 0 && w.tk_splits > 0) {
     // few rows of many candidates: the top-k split over S slices per row
-    TopkSplitParams tp;
+    TopkSplitParams tp{};
     uint8_t* lists = b + w.logits + w.part + w.ml + w.sigma;
     const size_t n_list = (size_t)batch * w.tk_splits * topk;
     tp.sigma = sigma;
@@ -495,6 +496,7 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
     tp.topk = topk;
     tp.window = window;
     tp.pos = kv_len - 1;
+    tp.pos_offset = 0;
     tp.cval = reinterpret_cast<float*>(lists);
     tp.cpos = reinterpret_cast<int32_t*>(lists + n_list * 4);
     tp.ccnt = reinterpret_cast<int32_t*>(lists + n_list * 8);
@@ -578,6 +580,96 @@ hs2_status swa_attn(const void* Q, const void* K, const void* V, int64_t q_start
   prof_begin(st);
   fa_fwd_kernel<D><<<fp.n_qtiles, FA_THREADS, FaLayout<D>::SMEM, st>>>(mQ, mK, mV, fp, ctx);
   return after_launch("fa_fwd_kernel", st);
+}
+
+// ---- context-sharded decode: one shard of every sequence's cache per GPU
+struct ShardWs {
+  size_t logits, part, sigma, lists, total;
+  int64_t ld;
+  int splits;      // key splits of the shard's full-attention pass
+  int tk_splits;   // slices of the shard's candidates
+};
+// Slices of a shard's candidates: the slices' lists must merge in one CTA.
+int shard_slices(int64_t n, int k) {
+  int64_t S = std::max<int64_t>(1, (n + TS_SLICE - 1) / TS_SLICE);
+  if (S > 1 && S * k > TS_CAP) S = std::max<int64_t>(1, TS_CAP / k);
+  return (int)S;
+}
+ShardWs shard_ws(int batch, int64_t shard_len, int Hq, int d, int topk) {
+  ShardWs w;
+  w.ld = round_up(shard_len, 64);
+  w.splits = (int)((shard_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit);
+  w.tk_splits = shard_slices(shard_len, topk);
+  w.logits = up256((size_t)batch * Hq * (size_t)w.ld * sizeof(float));
+  w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
+  w.sigma = up256((size_t)batch * (size_t)w.ld * sizeof(float));
+  w.lists = up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4));
+  w.total = w.logits + w.part + w.sigma + w.lists;
+  return w;
+}
+
+template <int D>
+hs2_status shard_attn(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
+                      int64_t shard_len, int64_t kv_stride, int Hq, float scale, float* ml_out, float* O_out,
+                      void* ws, int topk, cudaStream_t st, const DevCtx& ctx) {
+  const ShardWs w = shard_ws(batch, shard_len, Hq, D, topk);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  DecParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const uint8_t*>(K);
+  p.V = static_cast<const uint8_t*>(V);
+  p.ks = ks;
+  p.vs = vs;
+  p.kv_len = shard_len;
+  p.kv_stride = kv_stride;
+  p.H = Hq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.splits = w.splits;
+  p.per_split = kDecodeKeysPerSplit;
+  p.part = reinterpret_cast<float*>(b + w.logits);
+  p.logits = reinterpret_cast<float*>(b);
+  p.logit_ld = w.ld;
+  p.idx_offset = -1;
+  using L = DecLayout<D, true>;
+  auto k = decode_attn_kernel<D, true, true>;
+  hs2_status s = set_smem(k, L::SMEM);
+  if (s != HS2_OK) return s;
+  CUtensorMap mK, mV;
+  if ((s = make_map_u8_3d(&mK, K, D, (uint64_t)shard_len, (uint64_t)batch, D, (uint64_t)kv_stride * D, 128,
+                          L::CH)) != HS2_OK)
+    return s;
+  if ((s = make_map_u8_3d(&mV, V, D, (uint64_t)shard_len, (uint64_t)batch, D, (uint64_t)kv_stride * D, 128,
+                          L::CH)) != HS2_OK)
+    return s;
+  prof_begin(st);
+  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
+  if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
+  return launch_combine<D>(p.part, w.splits, Hq, nullptr, ml_out, batch, st, O_out);
+}
+
+template <int D>
+hs2_status shard_sparse(const DecParams& p0, int batch, int n_idx, int sms, float* ml_out, float* O_out, void* ws,
+                        cudaStream_t st, const DevCtx& ctx) {
+  DecParams p = p0;
+  int splits = sparse_decode_splits(batch, n_idx, sms);
+  p.splits = splits;
+  p.per_split = (n_idx + splits - 1) / splits;
+  p.part = static_cast<float*>(ws);
+  hs2_status s = launch_decode_parts<D>(p, batch, st, ctx);
+  if (s != HS2_OK) return s;
+  return launch_combine<D>(p.part, splits, p.H, nullptr, ml_out, batch, st, O_out);
+}
+
+template <int D>
+hs2_status launch_partial(bool finalize, const float* ml, int R, int shard, float* O32, float* ml_out,
+                          __nv_bfloat16* O, int batch, int H, cudaStream_t st) {
+  prof_begin(st);
+  if (finalize) {
+    partial_finalize_kernel<D><<<dim3(batch, H), D, 0, st>>>(ml, O32, O, H);
+    return after_launch("partial_finalize_kernel", st);
+  }
+  partial_merge_kernel<D><<<dim3(batch, H), D, 0, st>>>(ml, R, shard, O32, ml_out, H);
+  return after_launch("partial_merge_kernel", st);
 }
 
 }  // namespace
@@ -879,6 +971,7 @@ hs2_status hs2_sparse_attn_decode(const void* Q, const void* Kc, const void* Vc,
   p.splits = splits;
   p.per_split = (n_idx + splits - 1) / splits;
   p.O = static_cast<__nv_bfloat16*>(O);
+  p.idx_offset = -1;
   p.part = static_cast<float*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (splits > kMaxCluster) {
@@ -976,6 +1069,219 @@ hs2_status hs2_swa_attn_prefill(const void* Q, const void* K, const void* V, int
                                   workspace, st, ctx)
                   : swa_attn<128>(Q, K, V, q_start, Tq, kv_len, Hq, window, rope_dims, rope_base, softmax_scale, O,
                                   workspace, st, ctx);
+}
+
+hs2_status hs2_decode_shard_workspace(int batch, int64_t shard_len, int n_idx, int Hq, int d, int topk,
+                                      size_t* bytes) {
+  g_err[0] = 0;
+  HS2_CHECK(bytes, HS2_ERR_INVALID_ARG, "bytes is null");
+  HS2_CHECK(batch >= 1 && shard_len >= 1 && n_idx >= 1 && topk >= 1, HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  DevCtx ctx;
+  int sms = 0;
+  hs2_status s = device_ctx(&ctx, &sms);
+  if (s != HS2_OK) return s;
+  const size_t full = shard_ws(batch, shard_len, Hq, d, topk).total;
+  const int splits = sparse_decode_splits(batch, n_idx, sms);
+  const size_t sparse = up256((size_t)batch * splits * (32 + 16 * (size_t)d) * sizeof(float));
+  *bytes = std::max(full, sparse);
+  return HS2_OK;
+}
+
+hs2_status hs2_decode_shard_attn(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                                 const float* v_scale, int batch, int64_t shard_len, int64_t kv_stride_tokens,
+                                 int Hq, int d, int topk, float softmax_scale, float* ml_out, float* O_out,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(Q && Kc && Vc && k_scale && v_scale && ml_out && O_out, HS2_ERR_INVALID_ARG, "null pointer");
+  HS2_CHECK(aligned16(Q) && aligned16(Kc) && aligned16(Vc) && aligned4(k_scale) && aligned4(v_scale) &&
+                aligned4(ml_out) && aligned16(O_out),
+            HS2_ERR_INVALID_ARG, "misaligned pointer");
+  HS2_CHECK(batch >= 1 && shard_len >= 1 && kv_stride_tokens >= shard_len && topk >= 1, HS2_ERR_INVALID_ARG,
+            "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
+  HS2_CHECK(std::isfinite(softmax_scale) && softmax_scale > 0.f, HS2_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  HS2_CHECK((shard_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit <= kCombineMaxSplits, HS2_ERR_UNSUPPORTED,
+            "shard too long");
+  const size_t need = shard_ws(batch, shard_len, Hq, d, topk).total;
+  HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) && ws_bytes >= need,
+            HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? shard_attn<256>(Q, Kc, Vc, k_scale, v_scale, batch, shard_len, kv_stride_tokens, Hq,
+                                    softmax_scale, ml_out, O_out, workspace, topk, st, ctx)
+                  : shard_attn<128>(Q, Kc, Vc, k_scale, v_scale, batch, shard_len, kv_stride_tokens, Hq,
+                                    softmax_scale, ml_out, O_out, workspace, topk, st, ctx);
+}
+
+hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int batch, int64_t shard_len,
+                                       int64_t shard_offset, int64_t kv_len, int Hq, int d, int window, int topk,
+                                       const float* ml_global, void* cand, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(workspace && ml_global && cand, HS2_ERR_INVALID_ARG, "null pointer");
+  HS2_CHECK(aligned4(ml_global) && aligned4(cand), HS2_ERR_INVALID_ARG, "misaligned pointer");
+  const size_t n_cand = (size_t)batch * topk;
+  float* cand_val = static_cast<float*>(cand);
+  int32_t* cand_pos = static_cast<int32_t*>(cand) + n_cand;
+  int32_t* cand_cnt = static_cast<int32_t*>(cand) + 2 * n_cand;
+  HS2_CHECK(batch >= 1 && shard_len >= 1 && shard_offset >= 0 && shard_offset + shard_len <= kv_len &&
+                window >= 1 && topk >= 1,
+            HS2_ERR_INVALID_ARG, "bad sizes");
+  HS2_CHECK(window + topk <= 2048 && kv_len - window <= (1ll << 30), HS2_ERR_UNSUPPORTED, "index row too wide");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  const ShardWs w = shard_ws(batch, shard_len, Hq, d, topk);
+  HS2_CHECK(ws_bytes >= w.total && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0), HS2_ERR_WORKSPACE,
+            "the workspace of hs2_decode_shard_attn (%zu bytes) is needed", w.total);
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(workspace);
+  const float* logits = reinterpret_cast<const float*>(b);
+  float* sigma = reinterpret_cast<float*>(b + w.logits + w.part);
+  // this shard's candidates: global positions offset .. kv_len - 1 - window
+  const int64_t n = std::max<int64_t>(0, std::min<int64_t>(shard_len, kv_len - window - shard_offset));
+  if (n > 0) {
+    dim3 g((unsigned)((n + 255) / 256), (unsigned)batch);
+    prof_begin(st);
+    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml_global, Hq, n, sigma, w.ld);
+    if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
+  }
+  const int S = shard_slices(n, topk);
+  uint8_t* lists = b + w.logits + w.part + w.sigma;
+  const size_t n_list = (size_t)batch * S * topk;
+  TopkSplitParams tp{};
+  tp.sigma = sigma;
+  tp.ld = w.ld;
+  tp.n = n;
+  tp.splits = S;
+  tp.slice = round_up((n + S - 1) / S, 64);
+  tp.topk = topk;
+  tp.window = window;
+  tp.pos = kv_len - 1;
+  tp.pos_offset = shard_offset;
+  tp.idx = nullptr;
+  // one slice: its list is the shard's list; more: a merge of all of them into one
+  tp.cval = S == 1 ? cand_val : reinterpret_cast<float*>(lists);
+  tp.cpos = S == 1 ? cand_pos : reinterpret_cast<int32_t*>(lists + n_list * 4);
+  tp.ccnt = S == 1 ? cand_cnt : reinterpret_cast<int32_t*>(lists + n_list * 8);
+  tp.group = S;
+  tp.gval = cand_val;
+  tp.gpos = cand_pos;
+  tp.gcnt = cand_cnt;
+  HS2_CHECK(tp.slice <= TS_CAP && (int64_t)S * topk <= TS_CAP, HS2_ERR_UNSUPPORTED, "shard too long for its top-k");
+  if ((s = set_smem(topk_slice_kernel, TS_SMEM)) != HS2_OK) return s;
+  prof_begin(st);
+  topk_slice_kernel<<<dim3((unsigned)S, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+  if ((s = after_launch("topk_slice_kernel", st)) != HS2_OK) return s;
+  if (S > 1) {
+    if ((s = set_smem(topk_merge_kernel<false>, TS_SMEM)) != HS2_OK) return s;
+    prof_begin(st);
+    topk_merge_kernel<false><<<dim3(1u, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+    if ((s = after_launch("topk_merge_kernel", st)) != HS2_OK) return s;
+  }
+  return HS2_OK;
+}
+
+hs2_status hs2_decode_merge_candidates(const void* cand_all, int n_shards, int batch, int64_t kv_len, int window,
+                                       int topk, int32_t* idx, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(cand_all && idx, HS2_ERR_INVALID_ARG, "null pointer");
+  HS2_CHECK(aligned4(cand_all) && aligned4(idx), HS2_ERR_INVALID_ARG, "misaligned pointer");
+  HS2_CHECK(batch >= 1 && n_shards >= 1 && kv_len >= 1 && window >= 1 && topk >= 1, HS2_ERR_INVALID_ARG,
+            "bad sizes");
+  HS2_CHECK(n_shards <= 64 && (int64_t)n_shards * topk <= TS_CAP && window + topk <= 2048, HS2_ERR_UNSUPPORTED,
+            "at most 64 shards and %d candidates per row", TS_CAP);
+  DevCtx ctx;
+  hs2_status s = device_ctx(&ctx, nullptr);
+  if (s != HS2_OK) return s;
+  // shard q's block: scores [batch, k], positions [batch, k], lengths [batch]
+  const int64_t n_cand = (int64_t)batch * topk, P = 2 * n_cand + batch;
+  TopkSplitParams tp{};
+  tp.n = std::max<int64_t>(0, kv_len - window);
+  tp.splits = n_shards;
+  tp.topk = topk;
+  tp.window = window;
+  tp.pos = kv_len - 1;
+  tp.cval = const_cast<float*>(static_cast<const float*>(cand_all));
+  tp.cpos = const_cast<int32_t*>(static_cast<const int32_t*>(cand_all)) + n_cand;
+  tp.ccnt = const_cast<int32_t*>(static_cast<const int32_t*>(cand_all)) + 2 * n_cand;
+  tp.group = 0;
+  tp.idx = idx;
+  tp.v_row = topk;
+  tp.v_list = P;
+  tp.c_row = 1;
+  tp.c_list = P;
+  if ((s = set_smem(topk_merge_kernel<true>, TS_SMEM)) != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_begin(st);
+  topk_merge_kernel<true><<<(unsigned)batch, TS_THREADS, TS_SMEM, st>>>(tp, ctx);
+  return after_launch("topk_merge_kernel", st);
+}
+
+hs2_status hs2_sparse_decode_shard(const void* Q, const void* Kc, const void* Vc, const float* k_scale,
+                                   const float* v_scale, int batch, int64_t shard_len, int64_t kv_stride_tokens,
+                                   int64_t shard_offset, const int32_t* idx, int n_idx, int Hq, int d,
+                                   float softmax_scale, float* ml_out, float* O_out, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  hs2_status s = sparse_decode_args(Q, Kc, Vc, k_scale, v_scale, HS2_KV_FP8_E4M3, batch, shard_len, kv_stride_tokens,
+                                    idx, n_idx, Hq, d, softmax_scale, Q);
+  if (s != HS2_OK) return s;
+  HS2_CHECK(ml_out && O_out && aligned4(ml_out) && aligned16(O_out), HS2_ERR_INVALID_ARG, "ml_out / O_out");
+  HS2_CHECK(shard_offset >= 0, HS2_ERR_INVALID_ARG, "shard_offset must be >= 0");
+  DevCtx ctx;
+  int sms = 0;
+  if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
+  const int splits = sparse_decode_splits(batch, n_idx, sms);
+  const size_t need = up256((size_t)batch * splits * (32 + 16 * (size_t)d) * sizeof(float));
+  HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) && ws_bytes >= need,
+            HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
+  DecParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const uint8_t*>(Kc);
+  p.V = static_cast<const uint8_t*>(Vc);
+  p.ks = k_scale;
+  p.vs = v_scale;
+  p.idx = idx;
+  p.n_idx = n_idx;
+  p.kv_len = shard_len;
+  p.kv_stride = kv_stride_tokens;
+  p.H = Hq;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.idx_offset = shard_offset;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? shard_sparse<256>(p, batch, n_idx, sms, ml_out, O_out, workspace, st, ctx)
+                  : shard_sparse<128>(p, batch, n_idx, sms, ml_out, O_out, workspace, st, ctx);
+}
+
+hs2_status hs2_partial_merge(const float* ml_all, int n_shards, int shard, float* O32, float* ml_out, int batch,
+                             int Hq, int d, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(ml_all && O32 && ml_out && aligned4(ml_all) && aligned4(O32) && aligned4(ml_out), HS2_ERR_INVALID_ARG,
+            "null or misaligned pointer");
+  HS2_CHECK(batch >= 1 && batch <= 65535 && n_shards >= 1 && shard >= 0 && shard < n_shards, HS2_ERR_INVALID_ARG,
+            "bad sizes");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? launch_partial<256>(false, ml_all, n_shards, shard, O32, ml_out, nullptr, batch, Hq, st)
+                  : launch_partial<128>(false, ml_all, n_shards, shard, O32, ml_out, nullptr, batch, Hq, st);
+}
+
+hs2_status hs2_partial_finalize(const float* ml, const float* O32, void* O, int batch, int Hq, int d, void* stream) {
+  g_err[0] = 0;
+  HS2_CHECK(ml && O32 && O && aligned4(ml) && aligned4(O32) && aligned16(O), HS2_ERR_INVALID_ARG,
+            "null or misaligned pointer");
+  HS2_CHECK(batch >= 1 && batch <= 65535, HS2_ERR_INVALID_ARG, "bad batch");
+  HS2_CHECK(shape_ok(Hq, d), HS2_ERR_UNSUPPORTED, "Hq must be 8 or 16 and d 128 or 256");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 256 ? launch_partial<256>(true, ml, 1, 0, const_cast<float*>(O32), nullptr,
+                                        static_cast<__nv_bfloat16*>(O), batch, Hq, st)
+                  : launch_partial<128>(true, ml, 1, 0, const_cast<float*>(O32), nullptr,
+                                        static_cast<__nv_bfloat16*>(O), batch, Hq, st);
 }
 
 hs2_status hs2_device_status(void* stream) {

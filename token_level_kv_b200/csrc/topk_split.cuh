@@ -42,6 +42,7 @@ struct TopkSplitParams {
   int topk;              // k
   int window;
   int64_t pos;           // query position
+  int64_t pos_offset;    // added to the positions stored in the lists (a shard's first global position)
   float* cval;           // [batch, S, k] slice lists (scores)
   int32_t* cpos;         // [batch, S, k] (positions)
   int32_t* ccnt;         // [batch, S] list lengths
@@ -50,6 +51,10 @@ struct TopkSplitParams {
   int32_t* gpos;
   int32_t* gcnt;         // [batch, G]
   int32_t* idx;          // [batch, window + k]
+  // Where the final merge finds list s of row b when they are not the slice
+  // lists above (v_list > 0): scores and positions at (b * v_row + s * v_list)
+  // and its length at (b * c_row + s * c_list), in elements.
+  int64_t v_row, v_list, c_row, c_list;
 };
 
 // Exclusive prefix sum over the CTA; `total` gets the sum.
@@ -241,7 +246,7 @@ topk_slice_kernel(TopkSplitParams p, DevCtx ctx) {
     uint32_t x = __float_as_uint(src[c]);
     if (x > 0x7f800000u) x = 0u;
     p.cval[lo + at] = __uint_as_float(x);
-    p.cpos[lo + at] = (int32_t)(j0 + c);
+    p.cpos[lo + at] = (int32_t)(p.pos_offset + j0 + c);
     ++at;
   }
   if (threadIdx.x == 0) p.ccnt[b * p.splits + s] = (int32_t)total;
@@ -270,23 +275,26 @@ topk_merge_kernel(TopkSplitParams p, DevCtx ctx) {
   const int32_t* in_cnt = from_groups ? p.gcnt : p.ccnt;
   const int l0 = FINAL ? 0 : blockIdx.x * p.group;
   const int nl = FINAL ? n_lists_row : min(p.group, p.splits - l0);
+  const bool strided = FINAL && !from_groups && p.v_list > 0;
+  const int64_t v_row = strided ? p.v_row : (int64_t)n_lists_row * k, v_list = strided ? p.v_list : k;
+  const int64_t c_row = strided ? p.c_row : n_lists_row, c_list = strided ? p.c_list : 1;
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int s = 0; s < nl; ++s) {
       offs[s] = acc;
-      acc += in_cnt[b * n_lists_row + l0 + s];
+      acc += in_cnt[b * c_row + (l0 + s) * c_list];
     }
     offs[nl] = acc;
   }
   __syncthreads();
   const int M = offs[nl];
-  const int64_t lo = (b * n_lists_row + l0) * (int64_t)k;
+  const int64_t lo = b * v_row + l0 * v_list;       // list s of this CTA starts at lo + s * v_list
   // every list slot at once (independent loads); slot i of list s lands at offs[s] + i
   const int n_slot = nl * k;
 #pragma unroll 4
   for (int q = threadIdx.x; q < n_slot; q += TS_THREADS) {
     const int s = q / k, i = q - s * k;
-    if (i < offs[s + 1] - offs[s]) u[offs[s] + i] = __float_as_uint(in_val[lo + q]);
+    if (i < offs[s + 1] - offs[s]) u[offs[s] + i] = __float_as_uint(in_val[lo + s * v_list + i]);
   }
   __syncthreads();
   const int per = ts_per(M);
@@ -305,7 +313,7 @@ topk_merge_kernel(TopkSplitParams p, DevCtx ctx) {
     for (int c = c0; c < c1; ++c) {
       while (offs[s + 1] <= c) ++s;
       if (!u[c]) continue;
-      if (at < (uint32_t)k) out[W + at] = in_pos[lo + (int64_t)s * k + (c - offs[s])];
+      if (at < (uint32_t)k) out[W + at] = in_pos[lo + s * v_list + (c - offs[s])];
       ++at;
     }
     for (uint32_t i = total + threadIdx.x; i < (uint32_t)k; i += TS_THREADS) out[W + i] = -1;
@@ -316,7 +324,7 @@ topk_merge_kernel(TopkSplitParams p, DevCtx ctx) {
     for (int c = c0; c < c1; ++c) {
       while (offs[s + 1] <= c) ++s;
       if (!u[c]) continue;
-      const int64_t src = lo + (int64_t)s * k + (c - offs[s]);
+      const int64_t src = lo + s * v_list + (c - offs[s]);
       p.gval[olo + at] = in_val[src];
       p.gpos[olo + at] = in_pos[src];
       ++at;
