@@ -463,6 +463,7 @@ def run_ours(args, rank, world, dist):
         out["bridge"], bridged = bench_bridge(hs2, dev, stream, flush, peaks, peak_src)
         if not args.no_decode:
             out["decode_1m"] = bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged)
+            out["decode_1m_sharded"] = bench_sharded_decode(hs2, dev, stream, flush, args, bridged)
         del bridged
         torch.cuda.empty_cache()
     # ---------------- chunked prefill at 256k and the tiny launch-bound case
@@ -671,6 +672,104 @@ def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged
             "frac": byte_total / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": byte_total,
             "l2": "flushed before each step", "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
             "kernels": prof}
+
+
+class _OneProcessExchange:
+    """All shards in this process: the all-gather stacks, the all-reduce sums."""
+
+    def all_gather(self, local):
+        return torch.stack(local)
+
+    def all_reduce_sum(self, local):
+        total = torch.stack(local).sum(0)
+        for t in local:
+            t.copy_(total)
+
+
+def bench_sharded_decode(hs2, dev, stream, flush, args, bridged, R=4):
+    """The 1M-token decode of one cross-decoder layer (full + select, 3 sparse
+    layers) with each sequence's context split over R shards, against the
+    same layer on one GPU over the whole cache.  One GPU here: the shards run
+    one after another in this process, and what is timed for the sharded
+    case is shard 0's own calls (what each GPU of an R-GPU job runs between
+    its collectives); the exchanges are listed by size, not timed."""
+    import synth
+    from token_level_kv_b200 import sharded
+    caches, _, _ = bridged
+    c = synth.CONFIGS[5]
+    B, H, d, W, k, ns = c["B"], c["H"], c["d"], c["window"], c["topk"], c["n_sparse"]
+    N = BRIDGE["R"] // B
+    Q, Qsp = synth.bridged_decode_queries(B, H, d, 1, ns, seed=0, device=dev)[0]
+    K, V, ks, vs = caches[0]
+    Kc, Vc, ksc, vsc = K.view(B, N, d), V.view(B, N, d), ks.view(B, N), vs.view(B, N)
+    # one GPU, the whole cache
+    O = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    Os = torch.empty_like(O)
+    idx = torch.empty(B, W + k, dtype=torch.int32, device=dev)
+    ws = hs2.workspace(hs2.hs2_full_attn_select_workspace(hs2.KV_FP8_E4M3, B, 1, N, H, d, W, k), dev)
+    wss = hs2.workspace(hs2.hs2_sparse_attn_decode_workspace(B, W + k, H, d), dev)
+
+    def whole():
+        hs2.hs2_full_attn_select(Q, Kc, Vc, O, idx, ws, window=W, topk=k, k_scale=ksc, v_scale=vsc)
+        for Qs in Qsp:
+            hs2.hs2_sparse_attn_decode(Qs, Kc, Vc, ksc, vsc, idx, Os, wss)
+
+    # R shards in this process: one full step fills every exchanged buffer
+    sd = sharded.ShardedDecode(kv_len=N, n_shards=R, shards=list(range(R)), batch=B, Hq=H, d=d, window=W, topk=k,
+                               exchange=_OneProcessExchange(), device=dev)
+    parts = [tuple(t[:, o:o + n].contiguous() for t in (Kc, Vc, ksc, vsc)) for o, n in sd.bounds]
+    O_sh, idx_sh, _ = sd.step(Q, parts, Qsp)
+    s0, p0 = sd.local[0], parts[0]
+    ml_all = torch.stack([s.ml for s in sd.local])
+    cand_all = torch.stack([s.cand for s in sd.local])
+    mlg = torch.empty(B, H, 2, dtype=torch.float32, device=dev)
+    O0 = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    idx0 = torch.empty_like(idx)
+
+    def shard0():
+        hs2.hs2_decode_shard_attn(Q, *p0, s0.ml, s0.O32, s0.ws, topk=k, shard_len=s0.length)
+        hs2.hs2_partial_merge(ml_all, 0, s0.O32, mlg)
+        hs2.hs2_partial_finalize(mlg, s0.O32, O0)
+        hs2.hs2_decode_shard_candidates(s0.ws, mlg, s0.cand, batch=B, shard_len=s0.length, shard_offset=0,
+                                        kv_len=N, Hq=H, d=d, window=W, topk=k)
+        hs2.hs2_decode_merge_candidates(cand_all, idx0, kv_len=N, window=W, topk=k)
+        for Qs in Qsp:
+            hs2.hs2_sparse_decode_shard(Qs, *p0, idx_sh, s0.ml, s0.O32, s0.ws, shard_offset=0,
+                                        shard_len=s0.length)
+            hs2.hs2_partial_merge(ml_all, 0, s0.O32, mlg)
+            hs2.hs2_partial_finalize(mlg, s0.O32, O0)
+
+    res = {}
+    for name, fn in (("one_gpu", whole), ("shard", shard0)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        hs2.hs2_profile_enable(True)
+        t = timed_steps(fn, max(3, args.steps), flush, stream)
+        prof = per_kernel(hs2.hs2_profile_collect())
+        hs2.hs2_profile_enable(False)
+        res[name] = {"step_ms": statistics.median(t), "step_ms_cuda_graph": graph_step_ms(fn, max(3, args.steps),
+                                                                                          flush, stream),
+                     "kernels": prof}
+    whole()
+    agree = float((idx == idx_sh).float().mean())        # differ only where selection scores tie to rounding
+    if hs2.hs2_device_status() != 0:
+        raise RuntimeError("device status after the sharded decode")
+    n_coll = 3 * (1 + ns) + 1
+    ex_bytes = (1 + ns) * (R * 2 * B * H * 4 + B * H * d * 4) + R * hs2.candidates_numel(B, k) * 4
+    one, sh = res["one_gpu"], res["shard"]
+    del parts, sd
+    return {"workload": f"decode B={B} N={N} H={H} d={d}: one layer (full + select, {ns} sparse) over the FP8 "
+                        f"cache, the context split over {R} shards; shard 0 timed alone on this GPU",
+            "shards": R, "one_gpu_step_ms": one["step_ms"], "one_gpu_step_ms_cuda_graph": one["step_ms_cuda_graph"],
+            "per_shard_step_ms": sh["step_ms"], "per_shard_step_ms_cuda_graph": sh["step_ms_cuda_graph"],
+            "kernel_time_ratio": one["step_ms_cuda_graph"] / sh["step_ms_cuda_graph"],
+            "exchange": {"collectives_per_step": n_coll, "bytes_per_rank_per_step": ex_bytes,
+                         "kinds": "all-gather (m, l) and sum all-reduce O per layer, all-gather of the "
+                                  "candidate lists; not timed (one GPU)"},
+            "index_rows_agree_with_one_gpu": agree,
+            "kernels_one_gpu": one["kernels"], "kernels_shard": sh["kernels"],
+            "l2": "flushed before each step"}
 
 
 def bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args):
