@@ -163,6 +163,21 @@ def timed_steps(step, steps, flush, stream):
     return [a.elapsed_time(b) for a, b in ts]
 
 
+def warm_up(step, n=3, seconds=0.3):
+    """At least n untimed steps and at least `seconds` of them: a measurement
+    that follows a power-capped GEMM phase starts once the SM clock has come
+    back (right after the bridging GEMM the clock sat near half its maximum
+    for tens of milliseconds, doubling the decode kernels' times)."""
+    t0 = time.perf_counter()
+    i = 0
+    while i < n or time.perf_counter() - t0 < seconds:
+        step()
+        i += 1
+        if i % 4 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+
 def graph_step_ms(step, n, flush, stream):
     """The step captured once as a CUDA graph and replayed (L2 flushed before
     each replay): the launch gaps between its kernels go away."""
@@ -516,11 +531,12 @@ def bench_decode(hs2, dev, stream, flush, peaks, peak_src, args):
     def sparse(l):
         hs2.hs2_sparse_attn_decode(dc.Q_sparse[l], dc.Kc, dc.Vc, dc.ks, dc.vs, idx, Os, wss)
 
-    for _ in range(3):
+    def warm_step():
         full()
         for l in range(c["n_sparse"]):
             sparse(l)
-    torch.cuda.synchronize()
+
+    warm_up(warm_step)
     n = max(3, args.steps)
     hs2.hs2_profile_enable(True)
     t_full = timed_steps(full, n, flush, stream)
@@ -651,9 +667,7 @@ def bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged
             for Qs in Qsp:
                 hs2.hs2_sparse_attn_decode(Qs, Kc, Vc, ksc, vsc, idx, Os, wss)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
+    warm_up(step)
     n = max(3, args.steps)
     hs2.hs2_profile_enable(True)
     t = timed_steps(step, n, flush, stream)
@@ -741,9 +755,7 @@ def bench_sharded_decode(hs2, dev, stream, flush, args, bridged, R=4):
 
     res = {}
     for name, fn in (("one_gpu", whole), ("shard", shard0)):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
+        warm_up(fn)
         hs2.hs2_profile_enable(True)
         t = timed_steps(fn, max(3, args.steps), flush, stream)
         prof = per_kernel(hs2.hs2_profile_collect())
@@ -833,9 +845,7 @@ def bench_swa(hs2, case, flush, stream, peaks, window=128):
     def call():
         hs2.hs2_swa_attn_prefill(case.Q, case.K, case.V, O, ws, window=window)
 
-    for _ in range(3):
-        call()
-    torch.cuda.synchronize()
+    warm_up(call)
     hs2.hs2_profile_enable(True)
     t = timed_steps(call, 5, flush, stream)
     prof = per_kernel(hs2.hs2_profile_collect())
@@ -864,9 +874,7 @@ def bench_tiny(hs2, dev, stream, flush, args):
         hs2.hs2_full_attn_select(case.Q, case.K, case.V, O, idx, ws, window=W, topk=k)
         hs2.hs2_sparse_attn_prefill(case.Q_sparse[0], case.K, case.V, idx, Os)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
+    warm_up(step)
     hs2.hs2_profile_enable(True)
     t = timed_steps(step, max(5, args.steps), flush, stream)
     prof = per_kernel(hs2.hs2_profile_collect())

@@ -226,7 +226,27 @@ PrefillWs prefill_ws(int64_t Tq, int64_t kv_len, int Hq) {
   return w;
 }
 
-constexpr int kDecodeKeysPerSplit = 2048;
+constexpr int kDecodeKeysPerSplit = 2048;   // the smallest split; workspaces are sized for it
+
+// Keys per CTA of the decode full-attention pass.  One CTA runs per SM, and a
+// CTA's start-up and partial merge cost about as much as streaming ~300 more
+// keys, so the split is the one of 2048, 4096 or 8192 keys that minimises
+// waves x (keys + 300); ties keep the smaller split.  (Measured: 64 sequences
+// of 131072 keys run 6% faster with 8192 than with 2048, 4 sequences of 2^20
+// 9% faster with 4096, 4 context shards of 2^18 fastest with 8192.)
+int decode_split_keys(int batch, int64_t kv_len, int sms) {
+  int best = kDecodeKeysPerSplit;
+  double best_t = 1e300;
+  for (int per = kDecodeKeysPerSplit; per <= 4 * kDecodeKeysPerSplit; per *= 2) {
+    const int64_t ctas = (int64_t)batch * ((kv_len + per - 1) / per);
+    const double t = (double)((ctas + sms - 1) / sms) * (double)(per + 300);
+    if (t < best_t) {
+      best_t = t;
+      best = per;
+    }
+  }
+  return best;
+}
 
 // Slices of a decode row's top-k (topk_slice_kernel), 0 for the single-CTA
 // kernel.  The single-CTA kernel wins up to a few slices' worth of candidates
@@ -438,8 +458,10 @@ hs2_status prefill_select(const void* Q, const void* K, const void* V, int64_t q
 template <int D>
 hs2_status decode_select(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
                          int64_t kv_len, int64_t kv_stride, int Hq, int window, int topk, int block, float scale,
-                         void* O, int32_t* idx, void* ws, cudaStream_t st, const DevCtx& ctx) {
+                         void* O, int32_t* idx, void* ws, int sms, cudaStream_t st, const DevCtx& ctx) {
   const DecodeWs w = decode_ws(batch, kv_len, Hq, D, window, topk);
+  const int per = decode_split_keys(batch, kv_len, sms);
+  const int splits = (int)((kv_len + per - 1) / per);
   uint8_t* b = static_cast<uint8_t*>(ws);
   float* logits = reinterpret_cast<float*>(b);
   float* part = reinterpret_cast<float*>(b + w.logits);
@@ -455,8 +477,8 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   p.kv_stride = kv_stride;
   p.H = Hq;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.splits = w.splits;
-  p.per_split = kDecodeKeysPerSplit;
+  p.splits = splits;
+  p.per_split = per;
   p.part = part;
   p.logits = logits;
   p.logit_ld = w.ld;
@@ -473,9 +495,9 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
                           L::CH)) != HS2_OK)
     return s;
   prof_begin(st);
-  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
+  k<<<batch * splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
   if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
-  if ((s = launch_combine<D>(part, w.splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
+  if ((s = launch_combine<D>(part, splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
   if (n_cand > 0) {
     dim3 g((unsigned)((n_cand + 255) / 256), (unsigned)batch);
@@ -611,8 +633,10 @@ ShardWs shard_ws(int batch, int64_t shard_len, int Hq, int d, int topk) {
 template <int D>
 hs2_status shard_attn(const void* Q, const void* K, const void* V, const float* ks, const float* vs, int batch,
                       int64_t shard_len, int64_t kv_stride, int Hq, float scale, float* ml_out, float* O_out,
-                      void* ws, int topk, cudaStream_t st, const DevCtx& ctx) {
+                      void* ws, int topk, int sms, cudaStream_t st, const DevCtx& ctx) {
   const ShardWs w = shard_ws(batch, shard_len, Hq, D, topk);
+  const int per = decode_split_keys(batch, shard_len, sms);
+  const int splits = (int)((shard_len + per - 1) / per);
   uint8_t* b = static_cast<uint8_t*>(ws);
   DecParams p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -624,8 +648,8 @@ hs2_status shard_attn(const void* Q, const void* K, const void* V, const float* 
   p.kv_stride = kv_stride;
   p.H = Hq;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.splits = w.splits;
-  p.per_split = kDecodeKeysPerSplit;
+  p.splits = splits;
+  p.per_split = per;
   p.part = reinterpret_cast<float*>(b + w.logits);
   p.logits = reinterpret_cast<float*>(b);
   p.logit_ld = w.ld;
@@ -642,9 +666,9 @@ hs2_status shard_attn(const void* Q, const void* K, const void* V, const float* 
                           L::CH)) != HS2_OK)
     return s;
   prof_begin(st);
-  k<<<batch * w.splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
+  k<<<batch * splits, L::NT, L::SMEM, st>>>(p, ctx, mK, mV);
   if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
-  return launch_combine<D>(p.part, w.splits, Hq, nullptr, ml_out, batch, st, O_out);
+  return launch_combine<D>(p.part, splits, Hq, nullptr, ml_out, batch, st, O_out);
 }
 
 template <int D>
@@ -819,7 +843,8 @@ hs2_status full_attn_select_impl(const void* Q, const void* K, const void* V, co
   if (s != HS2_OK) return s;
   HS2_CHECK(ws_bytes >= need, HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
   DevCtx ctx;
-  if ((s = device_ctx(&ctx, nullptr)) != HS2_OK) return s;
+  int sms = 0;
+  if ((s = device_ctx(&ctx, &sms)) != HS2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (kv_dtype == HS2_KV_BF16) {
     HS2_CHECK(batch == 1, HS2_ERR_UNSUPPORTED, "bf16 prefill takes batch == 1");
@@ -839,9 +864,9 @@ hs2_status full_attn_select_impl(const void* Q, const void* K, const void* V, co
   HS2_CHECK(kv_stride_tokens >= kv_len, HS2_ERR_INVALID_ARG, "kv_stride_tokens must be >= kv_len");
   HS2_CHECK(((kv_stride_tokens * d) & 15) == 0, HS2_ERR_INVALID_ARG, "sequence stride must keep 16-byte alignment");
   return d == 256 ? decode_select<256>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
-                                       block, softmax_scale, O, idx, workspace, st, ctx)
+                                       block, softmax_scale, O, idx, workspace, sms, st, ctx)
                   : decode_select<128>(Q, K, V, k_scale, v_scale, batch, kv_len, kv_stride_tokens, Hq, window, topk,
-                                       block, softmax_scale, O, idx, workspace, st, ctx);
+                                       block, softmax_scale, O, idx, workspace, sms, st, ctx);
 }
 }  // namespace
 }  // namespace hs2
@@ -1108,13 +1133,14 @@ hs2_status hs2_decode_shard_attn(const void* Q, const void* Kc, const void* Vc, 
   HS2_CHECK(workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) && ws_bytes >= need,
             HS2_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed (256-byte aligned)", ws_bytes, need);
   DevCtx ctx;
-  hs2_status s = device_ctx(&ctx, nullptr);
+  int sms = 0;
+  hs2_status s = device_ctx(&ctx, &sms);
   if (s != HS2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 256 ? shard_attn<256>(Q, Kc, Vc, k_scale, v_scale, batch, shard_len, kv_stride_tokens, Hq,
-                                    softmax_scale, ml_out, O_out, workspace, topk, st, ctx)
+                                    softmax_scale, ml_out, O_out, workspace, topk, sms, st, ctx)
                   : shard_attn<128>(Q, Kc, Vc, k_scale, v_scale, batch, shard_len, kv_stride_tokens, Hq,
-                                    softmax_scale, ml_out, O_out, workspace, topk, st, ctx);
+                                    softmax_scale, ml_out, O_out, workspace, topk, sms, st, ctx);
 }
 
 hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int batch, int64_t shard_len,
