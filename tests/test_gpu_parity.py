@@ -247,9 +247,9 @@ def test_decode_select_fp8(hs2, B, N):
 
 @pytest.mark.parametrize("B,N", [(2, 140000), (1, 300000)])
 def test_decode_select_split_topk(hs2, B, N):
-    """Rows of more than 131072 candidates take the split top-k (exact top-k per
-    slice of about 32768, then one or two levels of merges of the slices'
-    lists): checked against the oracle."""
+    """Rows of more than 131072 candidates take the radix select over the whole
+    GPU (chunks of 8192 candidates adding to three digit histograms, then
+    a count and an ordered write): checked against the oracle."""
     case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=0, seed=18)
     O, idx = gpu_decode_select(case)
     ref = oracle.decode_select(case.Q, case.Kc, case.Vc, case.ks, case.vs, range(B), N, 128, 1024)
@@ -261,7 +261,7 @@ def test_decode_select_split_topk(hs2, B, N):
 
 def test_decode_split_topk_exact_ties_go_to_smaller_positions(hs2):
     """Every key identical: every candidate score is the same fp32 value, so the
-    selection must be positions 0..1023 exactly, across the slice boundaries."""
+    selection must be positions 0..1023 exactly, across the chunk boundaries."""
     B, N = 2, 300000
     case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=0, seed=19)
     case.Kc[:] = case.Kc[:, :1]

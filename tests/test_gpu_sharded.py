@@ -93,10 +93,11 @@ def test_sharded_decode_ties_go_to_smaller_positions(hs2):
         assert idx[b, :128].tolist() == list(range(N - 128, N))
 
 
-def test_sharded_decode_long_shards(hs2):
-    """Shards of more than 32768 candidates: each shard's top-k over several
-    slices and a merge, then the merge across shards."""
-    B, N = 1, 200000
+@pytest.mark.parametrize("B,N", [(1, 200000), (2, 300000)])
+def test_sharded_decode_long_shards(hs2, B, N):
+    """Shards of 100,000 candidates (each shard's top-k over several slices and
+    a merge) and of 150,000 (the radix select over the GPU, written as the
+    shard's list), then the merge across shards."""
     case = synth.make_decode_case(B, N, 16, 256, 128, 1024, n_sparse=1, seed=36)
     O, idx, outs = _run(hs2, case, 2)
     _check(case, O, idx, outs)

@@ -307,36 +307,42 @@ sparse_prefill_kernel(Attn16Params p, DevCtx ctx) {
   }
 }
 
-// Merge split partials of one (item, head) per CTA, one output dim per
-// thread: m = max m_s, l = sum l_s 2^(m_s-m), O = sum O_s 2^(m_s-m) / l.
-// Also stores (m, l) per head (log2 units) for the selection pass.  The
-// split factors are computed once, cooperatively, into shared memory, so the
-// O loop's loads are independent of one another (a full-attention pass over
-// 2^20 keys has 512 splits per sequence).
+// Merge split partials of one (item, head) per CTA: m = max m_s,
+// l = sum l_s 2^(m_s-m), O = sum O_s 2^(m_s-m) / l.  Also stores (m, l) per
+// head (log2 units) for the selection pass.  The split factors are computed
+// once, cooperatively, into shared memory; then G groups of D threads (one
+// output dim per thread) each sum every G-th split, so a sequence with
+// hundreds of splits has G times the loads in flight, and group 0 adds the
+// groups' sums in a fixed order.  G = 4 for many splits, 1 for few (where
+// the extra threads only add start-up).
 constexpr int kCombineMaxSplits = 1024;
+constexpr int kCombineManySplits = 64;
 // With O32 set, the merged O is written unnormalised (fp32, relative to m) for
 // a later merge across shards of the context, and O is not written.
-template <int D>
-__global__ void __launch_bounds__(D)
+template <int D, int G>
+__global__ void __launch_bounds__(D * G)
 attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, float* ml, float* O32) {
-  const int item = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
-  const int lane = c & 31, warp = c >> 5;
+  constexpr int NT = D * G;
+  const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int c = tid % D, grp = tid / D;
+  const int lane = tid & 31, warp = tid >> 5;
   constexpr int PS = 32 + 16 * D;                   // floats per partial
   __shared__ float fac[kCombineMaxSplits];
-  __shared__ float red[D / 32];
+  __shared__ float red[NT / 32];
+  __shared__ float osum[G > 1 ? G - 1 : 1][D];
   const float* base = part + (int64_t)item * splits * PS;
   float M = -INFINITY;
-  for (int s = c; s < splits; s += D) M = fmaxf(M, base[(int64_t)s * PS + h]);
+  for (int s = tid; s < splits; s += NT) M = fmaxf(M, base[(int64_t)s * PS + h]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) red[warp] = M;
   __syncthreads();
   M = red[0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+  for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
   float ls = 0.f;
-  for (int s = c; s < splits; s += D) {
+  for (int s = tid; s < splits; s += NT) {
     const float ms = base[(int64_t)s * PS + h];
     const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
     fac[s] = f;
@@ -348,17 +354,22 @@ attn16_combine_kernel(const float* part, int splits, int H, __nv_bfloat16* O, fl
   __syncthreads();
   float Ls = 0.f;
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) Ls += red[w];
+  for (int w = 0; w < NT / 32; ++w) Ls += red[w];
   const float* col = base + 32 + h * D + c;
   float acc0 = 0.f, acc1 = 0.f;
-  int s = 0;
+  int s = grp;
 #pragma unroll 4
-  for (; s + 1 < splits; s += 2) {
+  for (; s + G < splits; s += 2 * G) {
     acc0 += col[(int64_t)s * PS] * fac[s];
-    acc1 += col[(int64_t)(s + 1) * PS] * fac[s + 1];
+    acc1 += col[(int64_t)(s + G) * PS] * fac[s + G];
   }
   if (s < splits) acc0 += col[(int64_t)s * PS] * fac[s];
-  const float acc = acc0 + acc1;
+  float acc = acc0 + acc1;
+  if (grp > 0) osum[grp - 1][c] = acc;
+  __syncthreads();
+  if (grp != 0) return;
+#pragma unroll
+  for (int q = 0; q < G - 1; ++q) acc += osum[q][c];
   if (c == 0 && ml != nullptr) {
     const int64_t r = (int64_t)item * H + h;
     if (O32 != nullptr) {                           // a shard's partial: m, then l, each [items, H]
@@ -413,24 +424,49 @@ partial_finalize_kernel(const float* ml, const float* O32, __nv_bfloat16* O, int
 }
 
 // Decode selection score: sigma[b, j] = sum_h 2^(x_hj - m_h) / l_h for the
-// candidates j < n_cand (x: scaled logits in log2 units).
+// candidates j < n_cand (x: scaled logits in log2 units).  A thread takes four
+// consecutive candidates with 16-byte loads (rows start 16-byte aligned: the
+// leading dimensions are multiples of 64), the heads added in order.  With
+// `zero` set, n_zero words per row from zero + b * n_zero are cleared.
 __global__ void __launch_bounds__(256)
 decode_sigma_kernel(const float* logits, int64_t logit_ld, const float* ml, int H,
-                    int64_t n_cand, float* sigma, int64_t sigma_ld) {
+                    int64_t n_cand, float* sigma, int64_t sigma_ld, uint32_t* zero, int n_zero) {
   const int b = blockIdx.y;
   __shared__ float sM[16], sI[16];
+  if (zero != nullptr && blockIdx.x == 0)           // the row's top-k histograms, for the passes after this one
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[(int64_t)b * n_zero + i] = 0u;
   if (threadIdx.x < H) {
     sM[threadIdx.x] = ml[((int64_t)b * H + threadIdx.x) * 2];
     const float l = ml[((int64_t)b * H + threadIdx.x) * 2 + 1];
     sI[threadIdx.x] = 1.f / l;
   }
   __syncthreads();
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (j >= n_cand) return;
-  float acc = 0.f;
-  for (int h = 0; h < H; ++h)
-    acc += fast_exp2(logits[((int64_t)b * H + h) * logit_ld + j] - sM[h]) * sI[h];
-  sigma[(int64_t)b * sigma_ld + j] = acc;
+  const float* row = logits + (int64_t)b * H * logit_ld + j;
+  float* out = sigma + (int64_t)b * sigma_ld + j;
+  if (j + 4 <= n_cand) {
+    float4 x[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h)
+      if (h < H) x[h] = *reinterpret_cast<const float4*>(row + h * logit_ld);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < 16; ++h)
+      if (h < H) {
+        acc.x += fast_exp2(x[h].x - sM[h]) * sI[h];
+        acc.y += fast_exp2(x[h].y - sM[h]) * sI[h];
+        acc.z += fast_exp2(x[h].z - sM[h]) * sI[h];
+        acc.w += fast_exp2(x[h].w - sM[h]) * sI[h];
+      }
+    *reinterpret_cast<float4*>(out) = acc;
+    return;
+  }
+  for (int e = 0; e < 4 && j + e < n_cand; ++e) {
+    float acc = 0.f;
+    for (int h = 0; h < H; ++h) acc += fast_exp2(row[h * logit_ld + e] - sM[h]) * sI[h];
+    out[e] = acc;
+  }
 }
 
 }  // namespace hs2

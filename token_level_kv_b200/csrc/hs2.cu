@@ -23,6 +23,7 @@
 #include "rope_swa.cuh"
 #include "select_sigma.cuh"
 #include "topk.cuh"
+#include "topk_radix.cuh"
 #include "topk_split.cuh"
 #include "sparse_tc.cuh"
 
@@ -263,17 +264,52 @@ int topk_split_count(int64_t n, int k) {
 
 constexpr int kMergeGroup = 8;     // slice lists merged per CTA of the first merge level
 
+// Decode rows of more than this many candidates take the grid-wide radix
+// select (topk_radix.cuh): a few long rows otherwise leave most SMs idle.
+constexpr int64_t kRadixMinCand = 4 * TS_SLICE;
+int radix_chunks(int64_t n, int k) {
+  return (n > kRadixMinCand && n > k) ? (int)((n + RX_CHUNK - 1) / RX_CHUNK) : 0;
+}
+size_t radix_bytes(int batch, int chunks) {
+  return chunks ? up256((size_t)batch * RX_HIST * 4) + up256((size_t)batch * chunks * 8) : 0;
+}
+
+// The five radix-select launches over rp.chunks x batch CTAs (the histograms
+// were zeroed by decode_sigma_kernel).
+hs2_status launch_radix(const RadixParams& rp, int batch, cudaStream_t st, const DevCtx& ctx) {
+  const dim3 g((unsigned)rp.chunks, (unsigned)batch);
+  hs2_status s;
+  prof_begin(st);
+  radix_hist_kernel<0><<<g, RX_THREADS, 0, st>>>(rp, ctx);
+  if ((s = after_launch("radix_hist_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  radix_hist_kernel<1><<<g, RX_THREADS, 0, st>>>(rp, ctx);
+  if ((s = after_launch("radix_hist_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  radix_hist_kernel<2><<<g, RX_THREADS, 0, st>>>(rp, ctx);
+  if ((s = after_launch("radix_hist_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  radix_count_kernel<<<g, RX_THREADS, 0, st>>>(rp, ctx);
+  if ((s = after_launch("radix_count_kernel", st)) != HS2_OK) return s;
+  prof_begin(st);
+  radix_write_kernel<<<g, RX_THREADS, 0, st>>>(rp, ctx);
+  return after_launch("radix_write_kernel", st);
+}
+
 struct DecodeWs {
-  size_t logits, part, ml, sigma, lists, total;
+  size_t logits, part, ml, sigma, lists, radix, total;
   int64_t ld;
   int splits;        // key splits of the full-attention pass
   int tk_splits;     // slices of the top-k (0: single CTA per row)
+  int rx_chunks;     // chunks of the radix select (0: not used)
 };
 DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d, int window, int topk) {
   DecodeWs w;
   w.ld = round_up(kv_len, 64);
   w.splits = (int)((kv_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit);
-  w.tk_splits = topk_split_count(std::max<int64_t>(0, kv_len - window), topk);
+  w.rx_chunks = radix_chunks(std::max<int64_t>(0, kv_len - window), topk);
+  w.tk_splits = w.rx_chunks ? 0 : topk_split_count(std::max<int64_t>(0, kv_len - window), topk);
+  w.radix = radix_bytes(batch, w.rx_chunks);
   w.logits = up256((size_t)batch * Hq * (size_t)w.ld * sizeof(float));
   w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
   w.ml = up256((size_t)batch * Hq * 2 * sizeof(float));
@@ -282,7 +318,7 @@ DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d, int window, int top
   const int groups = w.tk_splits > kMergeGroup ? (w.tk_splits + kMergeGroup - 1) / kMergeGroup : 0;
   w.lists = up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4)) +
             up256((size_t)batch * groups * ((size_t)topk * 8 + 4));
-  w.total = w.logits + w.part + w.ml + w.sigma + w.lists;
+  w.total = w.logits + w.part + w.ml + w.sigma + w.lists + w.radix;
   return w;
 }
 
@@ -303,7 +339,10 @@ hs2_status launch_combine(const float* part, int splits, int H, __nv_bfloat16* O
                           cudaStream_t st, float* O32 = nullptr) {
   if (splits > kCombineMaxSplits) return fail(HS2_ERR_UNSUPPORTED, "%d split partials (at most %d)", splits, kCombineMaxSplits);
   prof_begin(st);
-  attn16_combine_kernel<D><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml, O32);
+  if (splits >= kCombineManySplits)
+    attn16_combine_kernel<D, 4><<<dim3(items, H), D * 4, 0, st>>>(part, splits, H, O, ml, O32);
+  else
+    attn16_combine_kernel<D, 1><<<dim3(items, H), D, 0, st>>>(part, splits, H, O, ml, O32);
   return after_launch("attn16_combine_kernel", st);
 }
 
@@ -499,11 +538,30 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   if ((s = after_launch("decode_attn_kernel", st)) != HS2_OK) return s;
   if ((s = launch_combine<D>(part, splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
+  const bool radix = block == 0 && w.rx_chunks > 0;
+  uint32_t* rx_hist = reinterpret_cast<uint32_t*>(b + w.logits + w.part + w.ml + w.sigma + w.lists);
   if (n_cand > 0) {
-    dim3 g((unsigned)((n_cand + 255) / 256), (unsigned)batch);
+    dim3 g((unsigned)((n_cand + 1023) / 1024), (unsigned)batch);
     prof_begin(st);
-    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld);
+    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml, Hq, n_cand, sigma, w.ld, radix ? rx_hist : nullptr,
+                                           RX_HIST);
     if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
+  }
+  if (radix) {
+    // few rows of many candidates: the radix select over the whole GPU
+    RadixParams rp{};
+    rp.sigma = sigma;
+    rp.ld = w.ld;
+    rp.n = n_cand;
+    rp.chunks = w.rx_chunks;
+    rp.topk = topk;
+    rp.window = window;
+    rp.pos = kv_len - 1;
+    rp.pos_offset = 0;
+    rp.hist = rx_hist;
+    rp.cnt = rx_hist + up256((size_t)batch * RX_HIST * 4) / 4;
+    rp.idx = idx;
+    return launch_radix(rp, batch, st, ctx);
   }
   if (block == 0 && w.tk_splits > 0) {
     // few rows of many candidates: the top-k split over S slices per row
@@ -606,10 +664,11 @@ hs2_status swa_attn(const void* Q, const void* K, const void* V, int64_t q_start
 
 // ---- context-sharded decode: one shard of every sequence's cache per GPU
 struct ShardWs {
-  size_t logits, part, sigma, lists, total;
+  size_t logits, part, sigma, lists, radix, total;
   int64_t ld;
   int splits;      // key splits of the shard's full-attention pass
   int tk_splits;   // slices of the shard's candidates
+  int rx_chunks;   // chunks of the radix select over them (0: the slices)
 };
 // Slices of a shard's candidates: the slices' lists must merge in one CTA.
 int shard_slices(int64_t n, int k) {
@@ -626,7 +685,9 @@ ShardWs shard_ws(int batch, int64_t shard_len, int Hq, int d, int topk) {
   w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
   w.sigma = up256((size_t)batch * (size_t)w.ld * sizeof(float));
   w.lists = up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4));
-  w.total = w.logits + w.part + w.sigma + w.lists;
+  w.rx_chunks = radix_chunks(shard_len, topk);
+  w.radix = radix_bytes(batch, w.rx_chunks);
+  w.total = w.logits + w.part + w.sigma + w.lists + w.radix;
   return w;
 }
 
@@ -1170,11 +1231,33 @@ hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int bat
   float* sigma = reinterpret_cast<float*>(b + w.logits + w.part);
   // this shard's candidates: global positions offset .. kv_len - 1 - window
   const int64_t n = std::max<int64_t>(0, std::min<int64_t>(shard_len, kv_len - window - shard_offset));
+  const int chunks = radix_chunks(n, topk);           // <= w.rx_chunks: n <= shard_len
+  uint32_t* rx_hist = reinterpret_cast<uint32_t*>(b + w.logits + w.part + w.sigma + w.lists);
   if (n > 0) {
-    dim3 g((unsigned)((n + 255) / 256), (unsigned)batch);
+    dim3 g((unsigned)((n + 1023) / 1024), (unsigned)batch);
     prof_begin(st);
-    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml_global, Hq, n, sigma, w.ld);
+    decode_sigma_kernel<<<g, 256, 0, st>>>(logits, w.ld, ml_global, Hq, n, sigma, w.ld,
+                                           chunks ? rx_hist : nullptr, RX_HIST);
     if ((s = after_launch("decode_sigma_kernel", st)) != HS2_OK) return s;
+  }
+  if (chunks) {
+    // a long shard: the radix select over the whole GPU, written as the shard's list
+    RadixParams rp{};
+    rp.sigma = sigma;
+    rp.ld = w.ld;
+    rp.n = n;
+    rp.chunks = chunks;
+    rp.topk = topk;
+    rp.window = window;
+    rp.pos = kv_len - 1;
+    rp.pos_offset = shard_offset;
+    rp.hist = rx_hist;
+    rp.cnt = rx_hist + up256((size_t)batch * RX_HIST * 4) / 4;
+    rp.idx = nullptr;
+    rp.lval = cand_val;
+    rp.lpos = cand_pos;
+    rp.lcnt = cand_cnt;
+    return launch_radix(rp, batch, st, ctx);
   }
   const int S = shard_slices(n, topk);
   uint8_t* lists = b + w.logits + w.part + w.sigma;
