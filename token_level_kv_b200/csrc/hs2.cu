@@ -249,20 +249,6 @@ int decode_split_keys(int batch, int64_t kv_len, int sms) {
   return best;
 }
 
-// Slices of a decode row's top-k (topk_slice_kernel), 0 for the single-CTA
-// kernel.  The single-CTA kernel wins up to a few slices' worth of candidates
-// per row (measured: 65 us against 134 us for 64 rows of 130944); longer rows
-// are cut so that each slice and the merged lists fit one CTA's shared memory.
-int topk_split_count(int64_t n, int k) {
-  if (n <= 4 * TS_SLICE) return 0;
-  int64_t S = (n + TS_SLICE - 1) / TS_SLICE;
-  if (S * k > TS_CAP) S = TS_CAP / k;
-  if (S < 2 || S > 64) return 0;
-  if (round_up((n + S - 1) / S, 64) > TS_CAP) return 0;
-  return (int)S;
-}
-
-constexpr int kMergeGroup = 8;     // slice lists merged per CTA of the first merge level
 
 // Decode rows of more than this many candidates take the grid-wide radix
 // select (topk_radix.cuh): a few long rows otherwise leave most SMs idle.
@@ -297,28 +283,22 @@ hs2_status launch_radix(const RadixParams& rp, int batch, cudaStream_t st, const
 }
 
 struct DecodeWs {
-  size_t logits, part, ml, sigma, lists, radix, total;
+  size_t logits, part, ml, sigma, radix, total;
   int64_t ld;
-  int splits;        // key splits of the full-attention pass
-  int tk_splits;     // slices of the top-k (0: single CTA per row)
-  int rx_chunks;     // chunks of the radix select (0: not used)
+  int splits;        // key splits of the full-attention pass (at the smallest split)
+  int rx_chunks;     // chunks of the radix select (0: one CTA per row)
 };
 DecodeWs decode_ws(int batch, int64_t kv_len, int Hq, int d, int window, int topk) {
   DecodeWs w;
   w.ld = round_up(kv_len, 64);
   w.splits = (int)((kv_len + kDecodeKeysPerSplit - 1) / kDecodeKeysPerSplit);
   w.rx_chunks = radix_chunks(std::max<int64_t>(0, kv_len - window), topk);
-  w.tk_splits = w.rx_chunks ? 0 : topk_split_count(std::max<int64_t>(0, kv_len - window), topk);
   w.radix = radix_bytes(batch, w.rx_chunks);
   w.logits = up256((size_t)batch * Hq * (size_t)w.ld * sizeof(float));
   w.part = up256((size_t)batch * w.splits * (32 + 16 * (size_t)d) * sizeof(float));
   w.ml = up256((size_t)batch * Hq * 2 * sizeof(float));
   w.sigma = up256((size_t)batch * (size_t)w.ld * sizeof(float));
-  // slice lists, then (with more than kMergeGroup slices) the first merge level's lists
-  const int groups = w.tk_splits > kMergeGroup ? (w.tk_splits + kMergeGroup - 1) / kMergeGroup : 0;
-  w.lists = up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4)) +
-            up256((size_t)batch * groups * ((size_t)topk * 8 + 4));
-  w.total = w.logits + w.part + w.ml + w.sigma + w.lists + w.radix;
+  w.total = w.logits + w.part + w.ml + w.sigma + w.radix;
   return w;
 }
 
@@ -539,7 +519,7 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
   if ((s = launch_combine<D>(part, splits, Hq, static_cast<__nv_bfloat16*>(O), ml, batch, st)) != HS2_OK) return s;
   const int64_t n_cand = std::max<int64_t>(0, kv_len - window);
   const bool radix = block == 0 && w.rx_chunks > 0;
-  uint32_t* rx_hist = reinterpret_cast<uint32_t*>(b + w.logits + w.part + w.ml + w.sigma + w.lists);
+  uint32_t* rx_hist = reinterpret_cast<uint32_t*>(b + w.logits + w.part + w.ml + w.sigma);
   if (n_cand > 0) {
     dim3 g((unsigned)((n_cand + 1023) / 1024), (unsigned)batch);
     prof_begin(st);
@@ -562,46 +542,6 @@ hs2_status decode_select(const void* Q, const void* K, const void* V, const floa
     rp.cnt = rx_hist + up256((size_t)batch * RX_HIST * 4) / 4;
     rp.idx = idx;
     return launch_radix(rp, batch, st, ctx);
-  }
-  if (block == 0 && w.tk_splits > 0) {
-    // few rows of many candidates: the top-k split over S slices per row
-    TopkSplitParams tp{};
-    uint8_t* lists = b + w.logits + w.part + w.ml + w.sigma;
-    const size_t n_list = (size_t)batch * w.tk_splits * topk;
-    tp.sigma = sigma;
-    tp.ld = w.ld;
-    tp.n = std::max<int64_t>(0, kv_len - window);
-    tp.splits = w.tk_splits;
-    tp.slice = round_up((tp.n + w.tk_splits - 1) / w.tk_splits, 64);   // 16-byte aligned slices
-    tp.topk = topk;
-    tp.window = window;
-    tp.pos = kv_len - 1;
-    tp.pos_offset = 0;
-    tp.cval = reinterpret_cast<float*>(lists);
-    tp.cpos = reinterpret_cast<int32_t*>(lists + n_list * 4);
-    tp.ccnt = reinterpret_cast<int32_t*>(lists + n_list * 8);
-    const int groups = w.tk_splits > kMergeGroup ? (w.tk_splits + kMergeGroup - 1) / kMergeGroup : 0;
-    uint8_t* glists = lists + up256((size_t)batch * w.tk_splits * ((size_t)topk * 8 + 4));
-    const size_t n_glist = (size_t)batch * groups * topk;
-    tp.group = groups ? kMergeGroup : 0;
-    tp.gval = reinterpret_cast<float*>(glists);
-    tp.gpos = reinterpret_cast<int32_t*>(glists + n_glist * 4);
-    tp.gcnt = reinterpret_cast<int32_t*>(glists + n_glist * 8);
-    tp.idx = idx;
-    if ((s = set_smem(topk_slice_kernel, TS_SMEM)) != HS2_OK) return s;
-    if ((s = set_smem(topk_merge_kernel<false>, TS_SMEM)) != HS2_OK) return s;
-    if ((s = set_smem(topk_merge_kernel<true>, TS_SMEM)) != HS2_OK) return s;
-    prof_begin(st);
-    topk_slice_kernel<<<dim3((unsigned)w.tk_splits, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
-    if ((s = after_launch("topk_slice_kernel", st)) != HS2_OK) return s;
-    if (groups) {
-      prof_begin(st);
-      topk_merge_kernel<false><<<dim3((unsigned)groups, (unsigned)batch), TS_THREADS, TS_SMEM, st>>>(tp, ctx);
-      if ((s = after_launch("topk_merge_kernel", st)) != HS2_OK) return s;
-    }
-    prof_begin(st);
-    topk_merge_kernel<true><<<(unsigned)batch, TS_THREADS, TS_SMEM, st>>>(tp, ctx);
-    return after_launch("topk_merge_kernel", st);
   }
   return launch_select(sigma, w.ld, kv_len - 1, 0, window, topk, block, idx, batch, st, ctx);
 }

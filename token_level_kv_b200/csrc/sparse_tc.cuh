@@ -7,9 +7,11 @@
 //
 // Design (sm_100a).  One persistent CTA per SM walks the query rows.
 //   * Eight producer warps gather the selected K and V rows with cp.async into
-//     a ring of 32 KB stages (128 keys x 128 dims, two 64-dim atom columns in
-//     the 128-byte swizzled layout the MMA reads); two lanes per 32-byte
-//     sector, so every request is a whole sector of one row.
+//     a ring whose stage is one tile's rows over the whole head dim (128 keys
+//     x d dims: 128-dim halves of two 64-dim atom columns in the 128-byte
+//     swizzled layout the MMA reads); two lanes per 32-byte sector, so every
+//     request is a whole sector of one row.  One commit per stage releases it
+//     (every 16 MMAs at d = 256).
 //   * One thread issues tcgen05.mma.  Per 128-key tile t it forms
 //     S^T_t = K_t Q^T (M = 128 keys, N = 16 heads, K = d) into TMEM columns
 //     [16t, 16t+16) of the row's S buffer; after the softmax it adds
@@ -28,9 +30,9 @@
 //     r+1's gather and Q K^T products.
 //   * P^T moves tile by tile through a 2-tile ring: the softmax writes tile t
 //     while the tensor cores multiply tile t-1, which leaves shared memory to
-//     a 6-stage gather ring (192 KB in flight).
+//     a 192 KB gather ring (3 stages at d = 256, 6 at d = 128).
 // Rows of up to 15 tiles (1920 keys): TMEM 2 x 240 + 32 columns (512 taken),
-// shared memory 6 x 32 KB ring + 2 x 4 KB P^T + 2 x 8 KB Q.
+// shared memory 192 KB ring + 2 x 4 KB P^T + 2 x 8 KB Q.
 #pragma once
 #include "attn16.cuh"
 #include "common.cuh"
@@ -42,12 +44,16 @@ struct StcLayout {
   static constexpr int NPROD = 8;                // producer warps (16 key rows of a stage each)
   static constexpr int MMA_WARP = 4 + NPROD;
   static constexpr int NT = (MMA_WARP + 1) * 32; // 4 softmax warps, the producers, 1 MMA warp
-  static constexpr int NSTG = 6;                 // ring stages
-  static constexpr int STAGE = 128 * 256;        // 128 keys x 128 dims bf16 (two 16 KB atom columns)
+  // a stage is one tile's K or V rows over the whole head dim: 128 keys x
+  // d/128 halves of 128 dims (two 16 KB atom columns each), so the MMA thread
+  // commits once per 16 (d = 256) or 8 (d = 128) MMAs
+  static constexpr int HALF = 128 * 256;         // bytes of one 128-dim half of a tile
+  static constexpr int STAGE = HALF * (D / 128);
+  static constexpr int NSTG = 6 / (D / 128);     // ring stages (192 KB)
   static constexpr int MAXT = 15;                // tiles of 128 keys per row
   static constexpr int SBUF = 16 * MAXT;         // TMEM columns of one S^T buffer
   static constexpr int OCOL = 2 * SBUF;          // O^T: 16 columns per half of d
-  static constexpr int HALVES = D / 128;         // stages per tile (K or V)
+  static constexpr int HALVES = D / 128;         // 128-dim halves per tile
   static constexpr int P_TILE = 16 * 256;        // P^T of one tile: 16 heads x 128 keys bf16
   static constexpr int NPS = 2;                  // P^T tiles in flight (softmax -> P V products)
   static constexpr int Q_BYTES = 16 * D * 2;     // 16 heads x d, D/64 atom columns of 2 KB
@@ -180,10 +186,10 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
             mypos = -1;
           }
           set_rows(reinterpret_cast<const uint8_t*>(p.K), mypos);
-          for (int c = 0; c < L::HALVES; ++c) {
+          {
             uint8_t* stg = acquire();
             if (!stg) { ok = false; break; }
-            if (t == 0 && c == 0) {
+            if (t == 0) {
               // the row's Q (16 heads; rows >= H zero) rides with the first stage
               const __nv_bfloat16* q = p.Q + row * p.H * D;
               for (int u = 32 * w + lane; u < 16 * D / 8; u += 32 * L::NPROD) {
@@ -193,7 +199,7 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
                            q + (h < p.H ? h : 0) * D + un * 8, h < p.H);
               }
             }
-            copy_rows(stg, c);
+            for (int c = 0; c < L::HALVES; ++c) copy_rows(stg + c * L::HALF, c);
             release();
           }
         }
@@ -206,12 +212,10 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
           nextpos = ldpos(irow, t + 1);
           if (mypos < -1 || mypos >= p.kv_len) mypos = -1;
           set_rows(reinterpret_cast<const uint8_t*>(p.V), mypos);
-          for (int c = 0; c < L::HALVES; ++c) {
-            uint8_t* stg = acquire();
-            if (!stg) { ok = false; break; }
-            copy_rows(stg, c);
-            release();
-          }
+          uint8_t* stg = acquire();
+          if (!stg) { ok = false; break; }
+          for (int c = 0; c < L::HALVES; ++c) copy_rows(stg + c * L::HALF, c);
+          release();
         }
       }
     }
@@ -237,21 +241,21 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
           const uint64_t dQ = umma_desc_sw128(smem_u32(sQ + (st & 1) * L::Q_BYTES), 16, 1024);
           const uint32_t sb = tmem + (st & 1) * L::SBUF;
           for (int t = 0; t < nT && ok; ++t) {
-            for (int c = 0; c < L::HALVES; ++c) {
-              if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
-              fence_proxy_async_smem();              // cp.async (generic) data -> tensor-core reads
-              tc_fence_after();
-              const uint64_t dK = dring0 + (uint64_t)(slot * (L::STAGE >> 4));
+            if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
+            fence_proxy_async_smem();                // cp.async (generic) data -> tensor-core reads
+            tc_fence_after();
+            const uint64_t dK = dring0 + (uint64_t)(slot * (L::STAGE >> 4));
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {           // 8 steps of 16 dims
-                const uint64_t ad = dK + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4);
+            for (int c = 0; c < L::HALVES; ++c)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {           // 8 steps of 16 dims per half
+                const uint64_t ad = dK + (uint64_t)((c * L::HALF + (k >> 2) * 16384 + (k & 3) * 32) >> 4);
                 const uint64_t bd = dQ + (uint64_t)((c * 4096 + (k >> 2) * 2048 + (k & 3) * 32) >> 4);
                 umma_bf16(sb + 16 * t, ad, bd, idS, (c | k) != 0 ? 1u : 0u);
               }
-              any = true;
-              umma_commit(&empty[slot]);
-              if (++slot == L::NSTG) { slot = 0; phase ^= 1; }
-            }
+            any = true;
+            umma_commit(&empty[slot]);
+            if (++slot == L::NSTG) { slot = 0; phase ^= 1; }
           }
           if (!ok) break;
           umma_commit(&s_full[st & 1]);
@@ -263,21 +267,21 @@ sparse_tc_kernel(Attn16Params p, DevCtx ctx) {
             if (!mbar_wait(&p_full[ps], (uint32_t)((pg / L::NPS) & 1), ctx)) { ok = false; break; }
             tc_fence_after();
             const uint64_t dP = dpt0 + (uint64_t)(ps * (L::P_TILE >> 4));
-            for (int c = 0; c < L::HALVES; ++c) {
-              if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
-              fence_proxy_async_smem();
-              tc_fence_after();
-              const uint64_t dV = dvring0 + (uint64_t)(slot * (L::STAGE >> 4));
+            if (!mbar_wait(&full[slot], phase, ctx)) { ok = false; break; }
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const uint64_t dV = dvring0 + (uint64_t)(slot * (L::STAGE >> 4));
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {           // 8 steps of 16 keys
-                const uint64_t ad = dV + (uint64_t)((k * 2048) >> 4);
+            for (int c = 0; c < L::HALVES; ++c)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {           // 8 steps of 16 keys per half
+                const uint64_t ad = dV + (uint64_t)((c * L::HALF + k * 2048) >> 4);
                 const uint64_t bd = dP + (uint64_t)(((k >> 2) * 2048 + (k & 3) * 32) >> 4);
                 umma_bf16(tmem + L::OCOL + 16 * c, ad, bd, idO, (t | k) != 0 ? 1u : 0u);
               }
-              umma_commit(&empty[slot]);
-              if (++slot == L::NSTG) { slot = 0; phase ^= 1; }
-            }
-            if (ok) umma_commit(&p_empty[ps]);
+            umma_commit(&empty[slot]);
+            if (++slot == L::NSTG) { slot = 0; phase ^= 1; }
+            umma_commit(&p_empty[ps]);
           }
           if (!ok) break;
           umma_commit(o_full);

@@ -1,6 +1,8 @@
-// Top-k of decode rows split over many CTAs (rows a4, a5 at decode): a few
-// sequences with up to 2^20 candidates each would leave one CTA per row doing
-// all the work, so each row is cut into S slices.
+// Top-k lists of slices of a row, and merges of such lists (rows a4, a5 of
+// the context-sharded decode): a shard's candidates are cut into S slices
+// whose exact top-k lists merge into the shard's list, and the shards' lists
+// merge into the index row.  (Long rows of the single-GPU decode take the
+// radix select of topk_radix.cuh instead.)
 //
 // Method: "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing"
 // (agihunt.info summary), KV Reuse paragraph -- the 128 most recent tokens
