@@ -414,8 +414,36 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
     if (threadIdx.x == 0) ncand = sb == 1 ? (uint32_t)n : m;
     __syncthreads();
     listed = true;
+    // the selects start from the sample's own pattern range [mn, mx], so
+    // near-equal scores spread over the bins from the first pass
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    {
+      const uint32_t cnt = sb == 1 ? (uint32_t)n : m;
+      for (uint32_t c = threadIdx.x; c < cnt; c += TK_THREADS) {
+        const uint32_t u = cval[c];
+        mn = min(mn, u);
+        mx = max(mx, u);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      const int warp = threadIdx.x >> 5;
+      if ((threadIdx.x & 31) == 0) {
+        hist[warp] = mn;                               // the bins are free until the select
+        hist[TK_NW + warp] = mx;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < TK_NW; ++w) {
+        mn = min(mn, hist[w]);
+        mx = max(mx, hist[TK_NW + w]);
+      }
+      __syncthreads();
+    }
     if (sb == 1) {
-      range_select(k, (uint32_t)n, 0u, 0x7f800000u, 0u);   // the whole row is the sample
+      range_select(k, (uint32_t)n, mn, mx, 0u);       // the whole row is the sample
     } else {
       const float ks = (float)k * (float)m / (float)n;
       const uint32_t rv = min(m, (uint32_t)(ks + 4.f * sqrtf(ks) + 8.f));
@@ -424,7 +452,7 @@ topk_select_kernel(TopkParams p, DevCtx ctx) {
         asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i));
       // the bound needs only the bin of the rv-th sample pattern, not the
       // pattern itself: one pass unless that bin is crowded
-      range_select(rv, m, 0u, 0x7f800000u, 16u);
+      range_select(rv, m, mn, mx, 16u);
       const uint32_t V = lo;
       collect(V);
       if (ncand >= k && ncand <= (uint32_t)TK_CAP) {
