@@ -130,3 +130,34 @@ def fp8_rule(codes, scales, exact, sabs):
     # x/scale is one fp32 division (2^-24 relative) of the accumulated value
     bad = np.abs(yg - np.clip(y, -448, 448)) > 0.5 * ulp + dlt / s[:, None] + 2.0 ** -22 * np.abs(y)
     return sbad, int(bad.sum())
+
+
+def plant_tie_keys(case, n_strong: int = 300, tie_every: int = 37, seed: int = 5):
+    """Decode case with a planted structure around the k-th score: per
+    sequence, n_strong keys (random candidate positions) far above every
+    random key, and one identical key at every tie_every-th other candidate
+    position, between the strong keys and the random ones.  The identical keys
+    tie exactly (same codes, same scale), so the selection takes all strong
+    keys and then the tied keys in position order, and the cut falls inside
+    the run of ties.  Returns {b: (strong positions, tie positions)}."""
+    import numpy as np
+    B, N, d = case.B, case.N, case.d
+    g = np.random.default_rng(seed)
+    n_cand = N - case.window
+    out = {}
+    for b in range(B):
+        qbar = case.Q[b].float().mean(dim=0)
+        u = qbar / qbar.norm()
+        strong = np.sort(g.choice(n_cand, n_strong, replace=False))
+        is_strong = np.zeros(n_cand, dtype=bool)
+        is_strong[strong] = True
+        ties = np.array([j for j in range(0, n_cand, tie_every) if not is_strong[j]], dtype=np.int64)
+        for pos, c in ((strong, 64.0), (ties, 40.0)):
+            v = (c * u).to(torch.bfloat16).float()
+            sc = v.abs().max() / 448.0
+            code = (v / sc).to(torch.float8_e4m3fn).view(torch.uint8)
+            idx = torch.as_tensor(pos)
+            case.Kc[b, idx] = code
+            case.ks[b, idx] = sc
+        out[b] = (strong, ties)
+    return out

@@ -272,6 +272,27 @@ def test_decode_split_topk_exact_ties_go_to_smaller_positions(hs2):
         assert idx[b, :128].tolist() == list(range(N - 128, N))
 
 
+def test_decode_radix_ties_inside_the_cut(hs2):
+    """Rows of 199,872 candidates (the radix select) with 300 strong keys and a
+    run of identical keys at every 37th other position: the selection is the
+    strong keys plus the first 724 tied keys in position order, a tie run that
+    crosses chunk boundaries and is cut inside (the ties taken are fewer than
+    the ties present); checked against the oracle exactly."""
+    from hs2_cases import plant_tie_keys
+    B, N, k = 2, 200000, 1024
+    case = synth.make_decode_case(B, N, 16, 256, 128, k, n_sparse=0, seed=21)
+    planted = plant_tie_keys(case)
+    O, idx = gpu_decode_select(case)
+    ref = oracle.decode_select(case.Q, case.Kc, case.Vc, case.ks, case.vs, range(B), N, 128, k)
+    for b in range(B):
+        strong, ties = planted[b]
+        want = np.sort(np.concatenate([strong, ties[:k - len(strong)]]))
+        assert np.array_equal(ref[b].idx[128:], want)                 # the oracle agrees with the construction
+        assert np.array_equal(idx[b, 128:].numpy(), want)
+        assert ties[k - len(strong) - 1] > 2 * 8192 and len(ties) > k - len(strong)   # across chunks, cut inside
+        assert max_abs(O[b].float().numpy(), ref[b].O) <= TOL_FP8
+
+
 def test_sparse_decode_many_sequences(hs2):
     """More sequences than SMs' worth of splits, kv_len below the row stride."""
     B, N = 70, 3000

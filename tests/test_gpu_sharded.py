@@ -113,3 +113,19 @@ def test_shard_calls_reject_bad_arguments(hs2):
         hs2.hs2_decode_merge_candidates(cand, torch.empty(1, 144, dtype=torch.int32, device="cuda"), kv_len=5000,
                                         window=128, topk=16)
     assert hs2.hs2_device_status() == 0
+
+
+def test_sharded_decode_ties_inside_the_cut(hs2):
+    """Two shards of 150,000 candidates each (the radix select writing the
+    shards' lists), strong keys and a run of exactly tied keys around the cut:
+    the merged selection is the strong keys plus the first tied keys in
+    position order across the shard boundary's lists."""
+    from hs2_cases import plant_tie_keys
+    B, N, k = 1, 300000, 1024
+    case = synth.make_decode_case(B, N, 16, 256, 128, k, n_sparse=0, seed=37)
+    planted = plant_tie_keys(case, n_strong=300, tie_every=400)
+    _, idx, _ = _run(hs2, case, 2)
+    strong, ties = planted[0]
+    want = np.sort(np.concatenate([strong, ties[:k - len(strong)]]))
+    assert ties[k - len(strong) - 1] > 150000 and len(ties) > k - len(strong)   # taken ties in both shards, cut inside
+    assert np.array_equal(idx[0, 128:].numpy(), want)
