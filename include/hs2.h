@@ -134,7 +134,7 @@ HS2_API hs2_status hs2_bridge_append(const void* hidden, int batch, int hidden_d
  *            Q bf16 [Tq, Hq, d]; K, V bf16 [kv_len, d]; k_scale/v_scale NULL.
  *            A long prefill may be issued in query chunks (q_start > 0) over
  *            the causal prefix (kv_len = q_start + Tq).
- *   decode : kv_dtype HS2_KV_FP8_E4M3, batch >= 1, Tq == 1,
+ *   decode : kv_dtype HS2_KV_FP8_E4M3, 1 <= batch <= 65535, Tq == 1,
  *            q_start == kv_len - 1 (the cache already holds the new token).
  *            Q bf16 [batch, Hq, d]; K, V uint8 [batch, kv_stride_tokens, d];
  *            k_scale, v_scale fp32 [batch, kv_stride_tokens]; key j of
@@ -339,7 +339,7 @@ HS2_API hs2_status hs2_partial_finalize(const float* ml, const float* O32, void*
  * scores fp32 [batch, topk], then global positions int32 [batch, topk], then
  * list lengths int32 [batch]; a row's list is its top min(topk, n) candidates
  * in ascending position (the order of hs2_full_attn_select: score
- * descending, ties to the smaller position).
+ * descending, ties to the smaller position).  1 <= batch <= 65535.
  */
 HS2_API hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int batch,
                                                int64_t shard_len, int64_t shard_offset, int64_t kv_len,

@@ -858,6 +858,7 @@ hs2_status full_attn_select_impl(const void* Q, const void* K, const void* V, co
                                           idx, workspace, st, ctx);
   }
   HS2_CHECK(kv_dtype == HS2_KV_FP8_E4M3, HS2_ERR_INVALID_ARG, "bad kv_dtype");
+  HS2_CHECK(batch <= 65535, HS2_ERR_UNSUPPORTED, "at most 65535 sequences per call");
   HS2_CHECK(Tq == 1 && q_start == kv_len - 1, HS2_ERR_UNSUPPORTED,
             "FP8 decode takes Tq == 1 with q_start == kv_len - 1");
   HS2_CHECK(k_scale && v_scale && aligned4(k_scale) && aligned4(v_scale), HS2_ERR_INVALID_ARG,
@@ -1154,7 +1155,7 @@ hs2_status hs2_decode_shard_candidates(void* workspace, size_t ws_bytes, int bat
   float* cand_val = static_cast<float*>(cand);
   int32_t* cand_pos = static_cast<int32_t*>(cand) + n_cand;
   int32_t* cand_cnt = static_cast<int32_t*>(cand) + 2 * n_cand;
-  HS2_CHECK(batch >= 1 && shard_len >= 1 && shard_offset >= 0 && shard_offset + shard_len <= kv_len &&
+  HS2_CHECK(batch >= 1 && batch <= 65535 && shard_len >= 1 && shard_offset >= 0 && shard_offset + shard_len <= kv_len &&
                 window >= 1 && topk >= 1,
             HS2_ERR_INVALID_ARG, "bad sizes");
   HS2_CHECK(window + topk <= 2048 && kv_len - window <= (1ll << 30), HS2_ERR_UNSUPPORTED, "index row too wide");
