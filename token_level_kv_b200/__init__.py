@@ -33,7 +33,7 @@ class Hs2Error(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m token_level_kv_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python token_level_kv_b200/build.py` "
                           "(nvcc, sm_100a); there is no fallback implementation")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, L, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
