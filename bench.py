@@ -313,6 +313,12 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
+    if args.sharded_nccl:
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        res = bench_sharded_nccl(hs2, dev, stream, lambda: flush_buf.zero_(), args, rank, world)
+        if rank == 0:
+            print(json.dumps({"decode_1m_sharded_nccl": res}), flush=True)
+        return
     if args.only_decode:
         flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
@@ -480,6 +486,10 @@ def run_ours(args, rank, world, dist):
             out["decode_1m"] = bench_bridged_decode(hs2, dev, stream, flush, peaks, peak_src, args, bridged)
             out["decode_1m_sharded"] = bench_sharded_decode(hs2, dev, stream, flush, args, bridged)
         del bridged
+        torch.cuda.empty_cache()
+    # ---------------- the 1M decode with the context split over the ranks (NCCL exchanges)
+    if dist and not args.no_decode:
+        out["decode_1m_sharded_nccl"] = bench_sharded_nccl(hs2, dev, stream, flush, args, rank, world)
         torch.cuda.empty_cache()
     # ---------------- chunked prefill at 256k and the tiny launch-bound case
     if not args.no_long:
@@ -784,6 +794,44 @@ def bench_sharded_decode(hs2, dev, stream, flush, args, bridged, R=4):
             "l2": "flushed before each step"}
 
 
+def bench_sharded_nccl(hs2, dev, stream, flush, args, rank, world, warm=20):
+    """One layer of the 1M-token decode (4 sequences of 2^20 tokens: full +
+    select, 3 sparse layers) with each sequence's context split over the
+    world's ranks, one shard per GPU, the exchanges over NCCL (all-gathers of
+    (m, l) and of the candidate lists, sum all-reduces of O): device time per
+    step, max over ranks.  Every rank runs the same fixed number of steps, so
+    the collectives pair up."""
+    import synth
+    from token_level_kv_b200 import sharded
+    c = synth.CONFIGS[5]
+    B, N, H, d, W, k, ns = c["B"], c["N"], c["H"], c["d"], c["window"], c["topk"], c["n_sparse"]
+    case = synth.make_decode_case(B, N, H, d, W, k, n_sparse=ns, seed=0, device=dev)
+    sd = sharded.ShardedDecode(kv_len=N, n_shards=world, shards=[rank], batch=B, Hq=H, d=d, window=W, topk=k,
+                               exchange=sharded.GroupExchange(), device=dev)
+    off, n = sd.bounds[rank]
+    cache = tuple(t[:, off:off + n].contiguous() for t in (case.Kc, case.Vc, case.ks, case.vs))
+    Q, Qs = case.Q, list(case.Q_sparse)
+    del case
+    torch.cuda.empty_cache()
+
+    def step():
+        sd.step(Q, [cache], Qs)
+
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    torch.distributed.barrier()
+    t = timed_steps(step, max(3, args.steps), flush, stream)
+    torch.distributed.barrier()
+    ms = reduce_max(statistics.median(t), dev)
+    if hs2.hs2_device_status() != 0:
+        raise RuntimeError("device status after the sharded decode")
+    return {"workload": f"decode B={B} N={N} H={H} d={d}: one layer (full + select, {ns} sparse) with the context "
+                        f"split over {world} ranks, exchanges over NCCL",
+            "shards": world, "shard_len": n, "step_ms": ms, "tok_s": B / (ms * 1e-3),
+            "l2": "flushed before each step", "timing": "CUDA events per step, median, max over ranks"}
+
+
 def bench_prefill_256k(hs2, dev, stream, peaks, peak_src, args):
     """The long chunked prefill: T = 262144, Zipf key norms, the full layer in
     32 query chunks of 8192 over the causal prefix, then 2 sparse layers over
@@ -907,6 +955,8 @@ def main():
     ap.add_argument("--decode-N", type=int, default=None, help="override the decode context (small profiling cases)")
     ap.add_argument("--only-decode", action="store_true", help="run the decode measurement only")
     ap.add_argument("--decode-B", type=int, default=None, help="override the decode batch (small profiling cases)")
+    ap.add_argument("--sharded-nccl", action="store_true",
+                    help="run only the context-sharded 1M decode over NCCL (also as a single rank)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     if args.decode_N:
@@ -925,12 +975,15 @@ def main():
         if rank == 0:
             run_reference(args)
         return
-    dist = world > 1
+    dist = world > 1 or args.sharded_nccl
     if dist:
         import datetime
         local = int(os.environ.get("LOCAL_RANK", "0"))
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")   # a single rank started without torchrun
+        os.environ.setdefault("MASTER_PORT", "29533")
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        torch.distributed.init_process_group("nccl", rank=rank, world_size=world,
+                                             timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
