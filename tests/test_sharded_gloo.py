@@ -94,3 +94,14 @@ def test_shard_bounds_tile_the_context():
         assert all(b[i][0] + b[i][1] == b[i + 1][0] for i in range(R - 1))
         assert all(n > 0 for _, n in b) and (kv < 64 * R or all(o % 64 == 0 for o, _ in b))
     assert np.array_equal(shard_bounds(1 << 20, 4), [(q << 18, 1 << 18) for q in range(4)])
+
+
+def test_shard_bounds_refuse_more_shards_than_positions():
+    import pytest
+    sys.path.insert(0, ROOT)
+    from token_level_kv_b200.sharded import shard_bounds
+    with pytest.raises(ValueError):
+        shard_bounds(3, 4)
+    with pytest.raises(ValueError):
+        shard_bounds(100, 0)
+    assert shard_bounds(5, 5) == [(i, 1) for i in range(5)]

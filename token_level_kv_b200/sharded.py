@@ -111,6 +111,8 @@ class ShardedDecode:
         shard i: codes uint8 [B, stride, d], scales fp32 [B, stride], local
         row r = global position offset + r.  O bf16 [B, H, d] and idx int32
         [B, window + topk] (global positions) are the same on every shard.
+        idx is this object's buffer: the next step overwrites it (the O
+        tensors are new each step).
     """
 
     def __init__(self, *, kv_len: int, n_shards: int, shards: list[int], batch: int, Hq: int, d: int,
