@@ -66,3 +66,37 @@ def test_cpu_tensors_are_refused_by_the_binding(hs2):
     x = torch.zeros(4, 16, 256, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         hs2.hs2_sparse_attn_prefill(x, x[0], x[0], torch.zeros(4, 8, dtype=torch.int32), x)
+
+
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    import shutil
+    import subprocess
+    src = tmp_path / "use_hs2.c"
+    src.write_text('#include "hs2.h"\nint main(void) { return (int)HS2_OK; }\n')
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not available")
+        lang = ["-x", "c++"] if cc == "g++" else []
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), *lang,
+                            "-c", str(src), "-o", str(tmp_path / f"use_{cc}.o")], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
+def test_shard_call_argument_checks_need_no_device(hs2):
+    lib = hs2.lib
+    n = ctypes.c_size_t(0)
+    # bad sizes and shapes are refused before any CUDA call
+    assert lib.hs2_decode_shard_workspace(0, 1000, 1152, 16, 256, 1024, ctypes.byref(n)) == 1
+    assert lib.hs2_decode_shard_workspace(4, 1000, 1152, 12, 256, 1024, ctypes.byref(n)) == 2
+    assert lib.hs2_decode_shard_attn(None, 16, 16, 16, 16, 4, 1000, 1000, 16, 256, 1024, 0.0625, 16, 16,
+                                     16, 1 << 20, None) == 1
+    assert lib.hs2_partial_merge(None, 2, 0, 16, 16, 4, 16, 256, None) == 1
+    assert lib.hs2_partial_merge(16, 2, 2, 16, 16, 4, 16, 256, None) == 1            # shard >= n_shards
+    assert lib.hs2_partial_finalize(16, 16, 16, 4, 12, 256, None) == 2               # Hq must be 8 or 16
+    assert lib.hs2_decode_merge_candidates(None, 2, 4, 10000, 128, 1024, 16, None) == 1
+    assert lib.hs2_decode_merge_candidates(16, 65, 4, 10000, 128, 1024, 16, None) == 2   # at most 64 shards
+    assert b"64" in lib.hs2_last_error()
+    assert lib.hs2_decode_shard_candidates(16, 1 << 20, 70000, 1000, 0, 1000, 16, 256, 128, 1024, 16, 16,
+                                           None) == 1                                    # batch > 65535
+    assert lib.hs2_sparse_decode_shard(16, 16, 16, 16, 16, 4, 1000, 1000, -1, 16, 1152, 16, 256, 0.0625, 16, 16,
+                                       16, 1 << 20, None) != 0                           # negative shard offset
